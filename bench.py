@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the Krea 2 backbone forward on B200 (sm_100a).
+
+A step is one full backbone forward (every step of the path: RoPE tables, time path, img_in,
+28 single-stream blocks, final layer) at 1024^2: batch 1, 512 text + 64x64 = 4096 image
+tokens, bf16 with fp32 residual. The metric is algorithmic TFLOP/s (GEMM FLOPs 2*M*N*K of the
+projections plus attention FLOPs 4*D*H*S*S_valid over valid keys). The same run also times
+the 1024^2 CFG block (batch 2, uncond row with 8 valid text tokens), per-kernel durations with
+CUDA events, an end-to-end pass through host buffers, and the CPU oracle on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Multi-GPU runs (torchrun, one rank per GPU) are replicas: each rank runs its own step with no
+data-path collective; time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import krea2_inputs as KI  # noqa: E402
+
+METRIC = "Krea2 block fwd bf16 TFLOP/s (% tensor peak); backbone ms/step at 1024²"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- work accounting
+
+def block_kernel_work(d: KI.Dims, B: int, T: int, N: int, lengths) -> dict:
+    """Algorithmic FLOPs (tensor kernels) or bytes (row kernels) of one block's launches."""
+    S = T + N
+    M = B * S
+    QC = d.qkvg_cols
+    valid = [(lengths[b] if T else 0) + N for b in range(B)]
+    return {
+        "modulation": {"bytes": B * 6 * d.C * 4 * 3},
+        "norm1": {"bytes": M * d.C * (4 + 2)},
+        "qkv_proj": {"flops": 2 * M * d.C * QC},
+        "attention": {"flops": 4 * d.D * d.H * sum(S * v for v in valid)},
+        "out_proj_resid": {"flops": 2 * M * d.HD * d.C},
+        "norm2": {"bytes": M * d.C * (4 + 2)},
+        "gate_up_swiglu": {"flops": 2 * M * d.C * 2 * d.F},
+        "down_proj_resid": {"flops": 2 * M * d.F * d.C},
+    }
+
+
+def block_flops(d, B, T, N, lengths) -> float:
+    return float(sum(v.get("flops", 0) for v in block_kernel_work(d, B, T, N, lengths).values()))
+
+
+def backbone_flops(d, B, T, N, lengths) -> float:
+    extra = 2 * B * (d.t_dim * d.C + d.C * d.C + d.C * 6 * d.C) + 2 * B * N * d.in_ch * d.C * 2
+    return d.n_layers * block_flops(d, B, T, N, lengths) + extra
+
+
+def oracle_block_flops(d, B, S, R, valid) -> float:
+    """FLOPs of one oracle block computing R sampled query rows per batch row (all keys)."""
+    M = B * S
+    kv = 2 * M * d.C * 2 * d.KVD
+    qg = 2 * B * R * d.C * 2 * d.HD
+    attn = 4 * d.D * d.H * R * sum(valid)
+    out = 2 * B * R * d.HD * d.C
+    mlp = 2 * B * R * d.C * 2 * d.F + 2 * B * R * d.F * d.C
+    return float(kv + qg + attn + out + mlp)
+
+
+def peaks() -> dict:
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p["bf16_tflops_sustained"], "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "flow_matching_stream_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernels."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_hash") != kernel_source_hash():
+        return None
+    return t.get("kernels", {}).get(kernel, {}).get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.ident = str(device_index)
+        try:
+            self.ident = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            pass
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", self.ident], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+class OracleSample:
+    """The CPU oracle (numpy fp32, fp64 softmax) on one block of the backbone workload, computing
+    `rows` sampled query rows over all keys. Inputs are generated once; run() is timed."""
+
+    def __init__(self, rows: int):
+        from oracle import krea2_oracle as O
+        self.O = O
+        wl = KI.backbone_1024()
+        self.d = d = wl.dims
+        self.wl = wl
+        self.h = KI.residual(d, wl.B, wl.S)
+        self.temb = KI.temb(d, wl.B)
+        self.w = KI.block_weights(d, 0)
+        self.c, self.s = O.rope_cos_sin(wl.positions(), d.axes, d.theta)
+        self.kv = O.key_valid_mask(wl.mask(), wl.B, wl.T, wl.N)
+        self.rows = rows
+        self.sel = np.linspace(0, wl.S - 1, rows).astype(int)
+        valid = [int(self.kv[b].sum()) for b in range(wl.B)]
+        self.flops = oracle_block_flops(d, wl.B, wl.S, rows, valid)
+
+    def run(self) -> float:
+        d = self.d
+        t0 = time.perf_counter()
+        self.O.block_forward(self.h, self.temb, self.w, self.c, self.s, self.kv, d.H, d.Hkv, d.D, d.eps,
+                             rows=self.sel, dtype=np.float32)
+        return time.perf_counter() - t0
+
+    def describe(self, seconds: float) -> str:
+        return (f"one block of the 1024^2 backbone workload (S=4608, C=6144), {self.rows} sampled query rows "
+                f"over all keys, numpy fp32 + fp64 softmax: {self.flops / 1e9:.0f} GFLOP in {seconds:.2f} s")
+
+
+def cpu_oracle_sample(rows: int = 512) -> dict:
+    o = OracleSample(rows)
+    dt = o.run()
+    return {"value": o.flops / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle", "sample": o.describe(dt)}
+
+
+# ----------------------------------------------------------------------------- native arm
+
+def run_native(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import flow_matching_stream_b200 as K2
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    warmup = max(args.warmup, 3)
+    wl = KI.backbone_1024()
+    d = wl.dims
+    B, T, N, S = wl.B, wl.T, wl.N, wl.S
+    dt = torch.bfloat16
+    gen = torch.Generator(device=dev).manual_seed(1234 + 0)  # same weights on every replica
+    blocks = [K2.BlockWeights.random(d, dt, dev, gen) for _ in range(d.n_layers)]
+    mw = K2.ModelWeights(KI.model_weights(d), blocks, dt, dev)
+
+    hidden_h = torch.from_numpy(KI.latents(d, B, N)).to(dt).pin_memory()
+    text_h = torch.from_numpy(KI.text_states(d, B, T)).to(dt).pin_memory()
+    pos_h = torch.from_numpy(wl.positions()).pin_memory()
+    mask_h = torch.from_numpy(wl.mask().astype(np.uint8)).pin_memory()
+    t_h = torch.from_numpy(KI.timesteps(B)).pin_memory()
+    vel_h = torch.empty(B, N, d.in_ch, dtype=dt).pin_memory()
+    hidden, text, pos, mask, tt = (x.to(dev) for x in (hidden_h, text_h, pos_h, mask_h, t_h))
+    vel = torch.empty(B, N, d.in_ch, device=dev, dtype=dt)
+    ws = torch.empty(K2.workspace_size(d, B, T, N, dt), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        K2.backbone_forward(d, B, T, N, hidden, text, pos, mask, tt, mw, vel, ws)
+
+    for _ in range(warmup):
+        step()
+    K2.check_device_error()
+
+    # ---- timed region: K backbone steps, inputs resident in HBM
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    l0 = K2.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = K2.launch_count() - l0
+    clk = clocks.stop()
+    K2.check_device_error()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    flops_step = backbone_flops(d, B, T, N, wl.lengths)
+    value = world * args.steps * flops_step / (ms_total / 1e3) / 1e12
+    ms_step = ms_total / args.steps
+
+    # ---- end to end through host buffers: H2D of the step's inputs, forward, D2H of velocity
+    h2d = sum(x.numel() * x.element_size() for x in (hidden_h, text_h, pos_h, mask_h, t_h))
+    d2h = vel_h.numel() * vel_h.element_size()
+
+    def e2e_step():
+        for dst, src in ((hidden, hidden_h), (text, text_h), (pos, pos_h), (mask, mask_h), (tt, t_h)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        vel_h.copy_(vel, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * args.steps * flops_step / (e2e_ms / 1e3) / 1e12
+
+    # ---- per-kernel durations (CUDA events on the launching stream) at the backbone's block shape
+    pk = peaks()
+    kernels = traced_block_kernels(K2, torch, d, B, T, N, wl.lengths, blocks[0], dev, reps=max(args.steps, 5))
+    dom = max((k for k in kernels if "tflops" in kernels[k]), key=lambda k: kernels[k]["ms"])
+    dk = kernels[dom]
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": dk["tflops"], "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": dk["tflops"] / pk["bf16_tflops_sustained"],
+                "traffic": recorded_traffic(dom), "peak_source": f"{pk['source']} sustained bf16 (kernel timed "
+                                                                   f"inside back-to-back blocks)",
+                "frac_of_burst": dk["tflops"] / pk["bf16_tflops"]}
+
+    # ---- the 1024^2 CFG block (batch 2: cond all 512 text valid, uncond 8 valid)
+    cfg = KI.block_1024_cfg()
+    cfg_res = time_block(K2, torch, cfg, dev, args.steps, warmup, pk)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": B, "text_tokens": T, "image_tokens": N, "seq_len": S,
+                   "layers": d.n_layers, "hidden": d.C, "heads": f"{d.H}q/{d.Hkv}kv x {d.D}",
+                   "intermediate": d.F, "weights": "random-init N(0,1)/sqrt(fan_in), seeded, ~12.2 B params bf16",
+                   "l2": "inputs larger than L2: 24 GB of block weights stream from HBM every step",
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "flops_per_step": flops_step},
+        "backbone_ms_per_step": ms_step,
+        "schedule_ms_forward_only": {"8_step": 8 * ms_step, "28_step": 28 * ms_step},
+        "pct_of_tensor_peak": {"burst": value / world / pk["bf16_tflops"],
+                               "sustained": value / world / pk["bf16_tflops_sustained"]},
+        "block_1024sq_cfg": cfg_res,
+        "kernels": kernels,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "ms_per_step": e2e_ms / args.steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": int(launches),
+        "gpu_launches_per_step": int(launches) // max(args.steps, 1),
+        "clocks": clk,
+        "peaks": pk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def traced_block_kernels(K2, torch, d, B, T, N, lengths, bw, dev, reps: int) -> dict:
+    S = T + N
+    pk = peaks()
+    h = torch.randn(B * S, d.C, device=dev)
+    temb = torch.randn(B, 6 * d.C, device=dev) * 0.5
+    pos = torch.from_numpy(KI.position_ids(T, int(np.sqrt(N)), N // int(np.sqrt(N)))).to(dev)
+    cs = torch.empty(S, d.D // 2, device=dev)
+    sn = torch.empty_like(cs)
+    K2.rope_tables(d, pos, cs, sn)
+    mask = torch.from_numpy(KI.mask_from_lengths(T, lengths).astype(np.uint8)).to(dev) if T else None
+    ws = torch.empty(K2.workspace_size(d, B, T, N, torch.bfloat16), dtype=torch.uint8, device=dev)
+    runs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(reps)]
+    for _ in range(3):
+        K2.block_forward(d, B, T, N, h, temb, bw, cs, sn, mask, ws)
+    for ev in runs:
+        K2.block_forward_traced(d, B, T, N, h, temb, bw, cs, sn, mask, ws, ev)
+    torch.cuda.synchronize()
+    K2.check_device_error()
+    work = block_kernel_work(d, B, T, N, lengths)
+    out = {}
+    for i, name in enumerate(K2.BLOCK_STEPS):
+        ms = float(np.mean([ev[i].elapsed_time(ev[i + 1]) for ev in runs]))
+        r = {"ms": ms}
+        if "flops" in work[name]:
+            r["tflops"] = work[name]["flops"] / (ms / 1e3) / 1e12
+            r["frac_sustained"] = r["tflops"] / pk["bf16_tflops_sustained"]
+        else:
+            r["gbs"] = work[name]["bytes"] / (ms / 1e3) / 1e9
+            r["frac_hbm"] = r["gbs"] / pk["hbm_gbs"]
+        out[name] = r
+    total = sum(v["ms"] for v in out.values())
+    for v in out.values():
+        v["share"] = v["ms"] / total
+    return out
+
+
+def time_block(K2, torch, wl: KI.Workload, dev, steps: int, warmup: int, pk: dict) -> dict:
+    d = wl.dims
+    gen = torch.Generator(device=dev).manual_seed(77)
+    bw = K2.BlockWeights.random(d, torch.bfloat16, dev, gen)
+    B, T, N, S = wl.B, wl.T, wl.N, wl.S
+    h = torch.randn(B * S, d.C, device=dev)
+    temb = torch.randn(B, 6 * d.C, device=dev) * 0.5
+    pos = torch.from_numpy(wl.positions()).to(dev)
+    cs = torch.empty(S, d.D // 2, device=dev)
+    sn = torch.empty_like(cs)
+    K2.rope_tables(d, pos, cs, sn)
+    mask = torch.from_numpy(wl.mask().astype(np.uint8)).to(dev)
+    ws = torch.empty(K2.workspace_size(d, B, T, N, torch.bfloat16), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        K2.block_forward(d, B, T, N, h, temb, bw, cs, sn, mask, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        K2.block_forward(d, B, T, N, h, temb, bw, cs, sn, mask, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    K2.check_device_error()
+    ms = e0.elapsed_time(e1) / steps
+    fl = block_flops(d, B, T, N, wl.lengths)
+    tf = fl / (ms / 1e3) / 1e12
+    kernels = traced_block_kernels(K2, torch, d, B, T, N, wl.lengths, bw, dev, reps=max(steps, 5))
+    return {"workload": wl.name, "ms_per_block": ms, "tflops": tf, "flops": fl,
+            "frac_burst": tf / pk["bf16_tflops"], "frac_sustained": tf / pk["bf16_tflops_sustained"],
+            "l2": "inputs larger than L2 (868 MB of block weights, ~1 GB of activations)",
+            "kernels": kernels}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int) -> None:
+    """The CPU oracle as the reference arm: each step is a bounded sample of the workload."""
+    if rank != 0:
+        return
+    warmup = max(args.warmup, 3)
+    o = OracleSample(rows=128)
+    for _ in range(warmup):
+        o.run()
+    times = [o.run() for _ in range(args.steps)]
+    el = float(sum(times))
+    value = o.flops * args.steps / el / 1e12
+    wl = KI.backbone_1024()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.B, "text_tokens": wl.T, "image_tokens": wl.N,
+                       "layers": wl.dims.n_layers},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+                             "kind": "oracle", "sample": o.describe(el / args.steps)},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    run_native(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,422 @@
+// Grouped-query flash attention of the Krea 2 block on the sm_100a tensor cores.
+//
+// Source: page "Diffusers 中的 Krea2Transformer2DModel … 架构全解", §四.3 (Krea2Attention /
+// Krea2AttnProcessor): q and k are RMS-normalised per head over head_dim, rotated by the 3-axis
+// RoPE, K/V heads are shared by H/Hkv = 4 consecutive query heads (the processor's
+// repeat_interleave order), the text padding mask removes keys, and the merged heads are
+// multiplied by sigmoid(to_gate(x)).
+//
+// Kernel layout (one CTA per (32 query positions, KV head j, batch row b)):
+//   * The 128-row MMA tile stacks the 4 query heads of KV head j: row r = 32*hl + p holds head
+//     4j+hl at position p0+p. One K/V tile in shared memory therefore serves all four heads
+//     (K/V are never copied per query head).
+//   * warp 0: TMA producer (Q once; K and V 128-key tiles, 2-stage ring). No cluster multicast.
+//   * warp 1: MMA issuer. S_i = Q K_iᵀ into one of two TMEM score buffers, O += P_{i-1} V_{i-1}
+//     into the TMEM output accumulator (V is the MN-major B operand, P the K-major A operand in
+//     shared memory).
+//   * warps 2..5: softmax, one thread per tile row (TMEM lane): row max from TMEM, lazy
+//     rescaling of O (only when the running max grows by more than 2^8), P = exp2 in bf16 to
+//     shared memory, final 1/l and sigmoid(gate) epilogue.
+//   * Key tiles whose 128 keys are all padded text are skipped entirely; partially padded
+//     tiles and the ragged end of the sequence are masked per key.
+// q and k arrive already RMS-normalised and rotated (the fused projection's epilogue or the
+// prep kernel below does that once per element); v and gate are raw projection columns.
+#include <cuda.h>
+
+#include "krea2_device.cuh"
+#include "krea2_internal.h"
+
+namespace krea2 {
+
+int make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t batches,
+                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+
+namespace {
+
+constexpr int AD = 128;          // head dim
+constexpr int AG = 4;            // query heads per KV head
+constexpr int QPOS = 32;         // query positions per CTA (x4 heads = 128 MMA rows)
+constexpr int KT = 128;          // keys per tile
+constexpr int KV_STAGES = 2;
+constexpr int ATT_THREADS = 192;
+constexpr int CHUNK_BYTES = 128 * 128;            // 128 rows x 64 bf16 (128 B) = 16 KB
+constexpr int Q_BYTES = 2 * CHUNK_BYTES;          // 32 KB
+constexpr int KV_TILE_BYTES = 2 * CHUNK_BYTES;    // 32 KB each for K and V
+constexpr int P_BYTES = 2 * CHUNK_BYTES;          // 32 KB
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + Q_BYTES;
+constexpr int OFF_V = OFF_K + KV_STAGES * KV_TILE_BYTES;
+constexpr int OFF_P = OFF_V + KV_STAGES * KV_TILE_BYTES;
+constexpr int ATT_SMEM = OFF_P + P_BYTES + 1024;
+constexpr int MAX_TILES = 512;   // S <= 65536
+constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, KT, 0, 0);
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AD, 0, 1);
+
+struct AttnCore {
+  int B, T, N, S, Hkv, HD;
+  const uint8_t* text_mask;
+  const __nv_bfloat16* gate;  // gate column block base (row stride g_stride)
+  long long g_stride;
+  __nv_bfloat16* out;         // (B*S, HD)
+  float scale_log2;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ bool key_valid(const AttnCore& p, int b, int t) {
+  if (t >= p.S) return false;
+  if (t < p.T && p.text_mask) return p.text_mask[(long)b * p.T + t] != 0;
+  return true;
+}
+
+__global__ void __launch_bounds__(ATT_THREADS, 1)
+    attn_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, AttnCore p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t k_full[KV_STAGES];
+  __shared__ __align__(8) uint64_t v_full[KV_STAGES];
+  __shared__ __align__(8) uint64_t kv_empty[KV_STAGES];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_full;
+  __shared__ __align__(8) uint64_t pv_done;
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  __shared__ int n_tiles;
+  __shared__ uint16_t tiles[MAX_TILES];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p0 = blockIdx.x * QPOS, j = blockIdx.y, b = blockIdx.z;
+  const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - smem_u32(smem_raw));
+
+  // ---- key tiles that hold at least one valid key (all-padded text tiles are skipped)
+  if (warp == 0) {
+    const int total = (p.S + KT - 1) / KT;
+    int count = 0;
+    for (int t0 = 0; t0 < total; t0 += 32) {
+      const int t = t0 + lane;
+      bool valid = false;
+      if (t < total) {
+        const int k0 = t * KT;
+        if (k0 + KT > p.T || !p.text_mask) {
+          valid = true;  // holds image keys (or no mask)
+        } else {
+          for (int k = k0; k < k0 + KT && !valid; ++k) valid = p.text_mask[(long)b * p.T + k] != 0;
+        }
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, valid);
+      if (valid) tiles[count + __popc(m & ((1u << lane) - 1u))] = (uint16_t)t;
+      count += __popc(m);
+    }
+    if (lane == 0) n_tiles = count;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(&p_full, 128);
+    mbar_init(&pv_done, 1);
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) tmem_alloc(&tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int n = n_tiles;
+  volatile int* abort = &abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&q_full, Q_BYTES);
+#pragma unroll
+      for (int hl = 0; hl < AG; ++hl)
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          tma_load_3d(base + OFF_Q + c * CHUNK_BYTES + hl * (QPOS * 128), &tmQ, &q_full,
+                      (j * AG + hl) * AD + c * 64, p0, b);
+      for (int i = 0; i < n; ++i) {
+        const int st = i % KV_STAGES;
+        const uint32_t ph = (i / KV_STAGES) & 1;
+        if (!mbar_wait(&kv_empty[st], ph ^ 1, abort)) break;
+        const int t0 = tiles[i] * KT;
+        mbar_arrive_expect_tx(&k_full[st], KV_TILE_BYTES);
+        tma_load_3d(base + OFF_K + st * KV_TILE_BYTES, &tmK, &k_full[st], j * AD, t0, b);
+        tma_load_3d(base + OFF_K + st * KV_TILE_BYTES + CHUNK_BYTES, &tmK, &k_full[st], j * AD + 64, t0, b);
+        mbar_arrive_expect_tx(&v_full[st], KV_TILE_BYTES);
+        tma_load_3d(base + OFF_V + st * KV_TILE_BYTES, &tmV, &v_full[st], j * AD, t0, b);
+        tma_load_3d(base + OFF_V + st * KV_TILE_BYTES + CHUNK_BYTES, &tmV, &v_full[st], j * AD + 64, t0, b);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t sq = smem_u32(base + OFF_Q);
+      const uint32_t sp = smem_u32(base + OFF_P);
+      bool issued = false;
+      auto issue_pv = [&](int i) -> bool {
+        // O += P_i V_i : A = P (K-major over keys), B = V (MN-major: d contiguous per key)
+        const int st = i % KV_STAGES;
+        if (!mbar_wait(&p_full, i & 1, abort)) return false;
+        if (!mbar_wait(&v_full[st], (i / KV_STAGES) & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t sv = smem_u32(base + OFF_V + st * KV_TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sp + (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, CHUNK_BYTES, 1024);
+          tc_mma_bf16(tmem + 256, ad, bd, IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&pv_done);
+        tc_commit(&kv_empty[st]);
+        return true;
+      };
+      if (mbar_wait(&q_full, 0, abort)) {
+        for (int i = 0; i < n; ++i) {
+          const int st = i % KV_STAGES;
+          if (!mbar_wait(&k_full[st], (i / KV_STAGES) & 1, abort)) break;
+          tc_fence_after();
+          const uint32_t sk = smem_u32(base + OFF_K + st * KV_TILE_BYTES);
+          const uint32_t d_s = tmem + (i & 1) * 128;
+#pragma unroll
+          for (int kk = 0; kk < AD / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
+            tc_mma_bf16(d_s, smem_desc_sw128(sq + off, 16, 1024), smem_desc_sw128(sk + off, 16, 1024), IDESC_QK,
+                        kk > 0 ? 1u : 0u);
+          }
+          issued = true;
+          tc_commit(&s_full[i & 1]);
+          if (i >= 1 && !issue_pv(i - 1)) break;
+        }
+        if (!*abort && n > 0) issue_pv(n - 1);
+      }
+      if (*abort && issued) {
+        tc_commit(&drain_bar);
+        unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+        }
+      }
+    }
+  } else {
+    // ---- softmax warps: quarter q of the tile = query head 4j+q, rows = 32 positions
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    uint8_t* prow = base + OFF_P + row * 128;
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int sb = i & 1;
+      if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const int t0 = tiles[i] * KT;
+      const bool partial = (t0 < p.T && p.text_mask) || (t0 + KT > p.S);
+      uint32_t vmask[4] = {~0u, ~0u, ~0u, ~0u};
+      if (partial) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) vmask[c] = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + c * 32 + lane));
+      }
+      const uint32_t sbase = tmem + lane_off + sb * 128;
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(sbase + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if ((vmask[c] >> e) & 1u) mx = fmaxf(mx, v[e]);
+      }
+      const float mnew = fmaxf(m, mx * sl2);
+      if (i >= 1 && !mbar_wait(&pv_done, (i - 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const bool grow = mnew > m + 8.0f;
+      if (__any_sync(0xffffffffu, grow)) {
+        const float alpha = grow ? ex2(m - mnew) : 1.f;  // m = -inf on the first tile -> 0
+        if (i >= 1) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_off + 256 + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tmem + lane_off + 256 + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+        if (grow) {
+          l *= alpha;
+          m = mnew;
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(sbase + c * 32, v);
+        float pr[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          pr[e] = ((vmask[c] >> e) & 1u) ? ex2(v[e] * sl2 - m) : 0.f;
+          l += pr[e];
+        }
+        // keys 32c..32c+31 -> chunk c/2, 16-byte granules 4*(c%2)..+3, 128-byte swizzle
+        uint8_t* chunk = prow + (c >> 1) * CHUNK_BYTES;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int gran = (c & 1) * 4 + g;
+          uint4 w;
+          w.x = pack_bf16x2(pr[g * 8 + 0], pr[g * 8 + 1]);
+          w.y = pack_bf16x2(pr[g * 8 + 2], pr[g * 8 + 3]);
+          w.z = pack_bf16x2(pr[g * 8 + 4], pr[g * 8 + 5]);
+          w.w = pack_bf16x2(pr[g * 8 + 6], pr[g * 8 + 7]);
+          *reinterpret_cast<uint4*>(chunk + ((gran ^ (row & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full);
+    }
+    if (ok && n > 0 && mbar_wait(&pv_done, (n - 1) & 1, abort)) {
+      tc_fence_after();
+      const int pos = p0 + lane;
+      const int h = j * AG + quarter;
+      const bool row_ok = pos < p.S;
+      const long grow_idx = (long)b * p.S + pos;
+      const float inv_l = 1.f / l;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_off + 256 + c * 32, o);
+        if (row_ok) {
+          const uint4* gp = reinterpret_cast<const uint4*>(p.gate + grow_idx * p.g_stride + h * AD + c * 32);
+          uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 gv = __ldg(gp + q);
+            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+            uint32_t ow[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a = o[q * 8 + 2 * e] * inv_l * sigmoid_f(bf16_lo(gw[e]));
+              const float bb = o[q * 8 + 2 * e + 1] * inv_l * sigmoid_f(bf16_hi(gw[e]));
+              ow[e] = pack_bf16x2(a, bb);
+            }
+            op[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (abort_flag) {
+    unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 1000000ull) {
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Raw projection -> RMS-normalised, rotated q and k (bf16), one warp per (row, head).
+// dst row layout: [q heads (H*D) | k heads (Hkv*D)].
+__global__ void __launch_bounds__(256) qk_prep_kernel(const __nv_bfloat16* __restrict__ src, long long src_stride,
+                                                      int S, int H, int Hkv, float eps,
+                                                      const float* __restrict__ qw, const float* __restrict__ kw,
+                                                      const float* __restrict__ cs, const float* __restrict__ sn,
+                                                      long rows, __nv_bfloat16* __restrict__ dst) {
+  const long gw = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int heads = H + Hkv;
+  if (gw >= rows * heads) return;
+  const long row = gw / heads;
+  const int hh = (int)(gw % heads);
+  const int pos = (int)(row % S);
+  const bool is_q = hh < H;
+  const float* w = is_q ? qw : kw;
+  const __nv_bfloat16* x = src + row * src_stride + (long)hh * AD + lane * 4;
+  const uint2 raw = *reinterpret_cast<const uint2*>(x);
+  float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+  const float ss = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
+  const float r = rsqrtf(ss / (float)AD + eps);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] *= r * (1.f + w[lane * 4 + e]);
+  const float c0 = cs[(long)pos * (AD / 2) + lane * 2], s0 = sn[(long)pos * (AD / 2) + lane * 2];
+  const float c1 = cs[(long)pos * (AD / 2) + lane * 2 + 1], s1 = sn[(long)pos * (AD / 2) + lane * 2 + 1];
+  const float y0 = v[0] * c0 - v[1] * s0, y1 = v[1] * c0 + v[0] * s0;
+  const float y2 = v[2] * c1 - v[3] * s1, y3 = v[3] * c1 + v[2] * s1;
+  uint2 o;
+  o.x = pack_bf16x2(y0, y1);
+  o.y = pack_bf16x2(y2, y3);
+  *reinterpret_cast<uint2*>(dst + row * (long)(heads * AD) + (long)hh * AD + lane * 4) = o;
+}
+
+}  // namespace
+
+KREA2_DEFINE_ERROR_READER(take_device_error_attention)
+
+bool attention_tc_supported(int D, int H, int Hkv) { return D == AD && Hkv > 0 && H == AG * Hkv; }
+
+int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(attn_gqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
+        cudaSuccess)
+      return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(attention) failed");
+    attr_done = true;
+  }
+  const int S = a.T + a.N;
+  if ((S + KT - 1) / KT > MAX_TILES) return set_error(KREA2_ERR_UNSUPPORTED, "sequence longer than %d", MAX_TILES * KT);
+  CUtensorMap tq, tk, tv;
+  int rc;
+  if ((rc = make_tmap_bf16_3d(&tq, a.q, (uint64_t)a.H * AD, S, a.B, a.q_stride, 64, QPOS))) return rc;
+  if ((rc = make_tmap_bf16_3d(&tk, a.k, (uint64_t)a.Hkv * AD, S, a.B, a.k_stride, 64, KT))) return rc;
+  if ((rc = make_tmap_bf16_3d(&tv, a.v, (uint64_t)a.Hkv * AD, S, a.B, a.v_stride, 64, KT))) return rc;
+  AttnCore p{};
+  p.B = a.B; p.T = a.T; p.N = a.N; p.S = S; p.Hkv = a.Hkv; p.HD = a.H * AD;
+  p.text_mask = a.text_mask;
+  p.gate = reinterpret_cast<const __nv_bfloat16*>(a.g);
+  p.g_stride = a.g_stride;
+  p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)AD);
+  dim3 grid((S + QPOS - 1) / QPOS, a.Hkv, a.B);
+  attn_gqa_tc_kernel<<<grid, ATT_THREADS, ATT_SMEM, stream>>>(tq, tk, tv, p);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
+  return KREA2_OK;
+}
+
+int launch_qk_prep(const void* qkvg, long long stride, int B, int S, int H, int Hkv, float eps, const float* qw,
+                   const float* kw, const float* cs, const float* sn, void* dst, cudaStream_t stream) {
+  const long rows = (long)B * S;
+  const long warps = rows * (H + Hkv);
+  qk_prep_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(qkvg), stride, S, H, Hkv, eps, qw, kw, cs, sn, rows,
+      reinterpret_cast<__nv_bfloat16*>(dst));
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "qk_prep launch failed: %s", cudaGetErrorString(e));
+  return KREA2_OK;
+}
+
+}  // namespace krea2

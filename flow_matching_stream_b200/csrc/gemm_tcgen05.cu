@@ -1,0 +1,448 @@
+// Dense bf16 projections of the Krea 2 block on the sm_100a tensor cores (tcgen05 + TMEM),
+// fed by TMA: out = A · Wᵀ with A (M, K) and W (N, K) both K-major (row-major, K contiguous).
+//
+// Used for the block's four linears (page "Diffusers 中的 Krea2Transformer2DModel … 架构全解",
+// §四.2 block and §四.3 attention): the fused [to_q | to_k | to_v | to_gate] projection, to_out
+// with the gated residual, the SwiGLU gate/up projection with silu(gate)*up, and the down
+// projection with the second gated residual.
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: A tile 128x64 and W tile BNx64 per stage, 128-byte swizzle,
+//               STAGES-deep ring guarded by full/empty mbarriers. No cluster multicast.
+//   warp 1      allocates TMEM (2 accumulators x BN fp32 columns) and issues tcgen05.mma
+//               (M=128, N=BN, K=16) from one thread; tcgen05.commit frees smem stages and
+//               signals a finished accumulator.
+//   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane), reads 32 columns
+//               at a time with tcgen05.ld and applies the fused epilogue, while the MMA warp
+//               already accumulates the next tile into the other TMEM buffer.
+// Tiles are visited in groups of GROUP_M row-tiles so that concurrently running CTAs share
+// W and A tiles through L2.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "krea2_device.cuh"
+#include "krea2_internal.h"
+
+namespace krea2 {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int GROUP_M = 16;
+constexpr int GEMM_THREADS = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+  static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN=256) or 16 KB (BN=128)
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+  static constexpr int TMEM_COLS = 2 * BN;                         // double-buffered fp32
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+};
+
+struct TileMap {
+  int tiles_m, tiles_n;
+  __device__ __forceinline__ void map(int t, int& mt, int& nt) const {
+    int per_group = GROUP_M * tiles_n;
+    int g = t / per_group;
+    int first_m = g * GROUP_M;
+    int gsize = min(tiles_m - first_m, GROUP_M);
+    int local = t - g * per_group;
+    mt = first_m + local % gsize;
+    nt = local / gsize;
+  }
+};
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - smem_u32(smem_raw));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(&tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  volatile int* abort = &abort_flag;
+
+  const TileMap tm{p.tiles_m, p.tiles_n};
+  const int total = p.tiles_m * p.tiles_n;
+  const int nk = p.K / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        int mt, nt;
+        tm.map(t, mt, nt);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort)) goto producer_done;
+          uint8_t* sa = base + stage * Cfg::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(sa, &tmA, &full_bar[stage], kb * BK, mt * BM);
+          tma_load_2d(sa + Cfg::A_BYTES, &tmB, &full_bar[stage], kb * BK, nt * BN);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    producer_done:;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int local = 0;
+      bool issued = false;
+      for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(base + stage * Cfg::STAGE_BYTES);
+          const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(sa + k * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + k * 32, 16, 1024);
+            tc_mma_bf16(d_tmem, ad, bd, Cfg::IDESC, (kb | k) != 0);
+          }
+          issued = true;
+          tc_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull_bar[acc]);
+      }
+      if (*abort && issued) {
+        // let every MMA already issued finish before TMEM is released
+        tc_commit(&drain_bar);
+        mbar_wait(&drain_bar, 0, &abort_flag /* already set: bounded by the timer below */);
+        unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < WAIT_LIMIT_NS) {
+        }
+      }
+    }
+  } else {
+    // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
+    const int quarter = warp & 3;
+    int local = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
+      int mt, nt;
+      tm.map(t, mt, nt);
+      const int acc = local & 1;
+      const uint32_t acc_phase = (local >> 1) & 1;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, abort)) break;
+      tc_fence_after();
+      const int row = mt * BM + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+
+      if constexpr (EPI == EPI_STORE) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + (size_t)nt * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 w;
+              w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+              w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+              w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+              w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+              dst[q] = w;
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU) {
+        // interleaved 64-row groups: columns [128g, 128g+64) gate, [128g+64, 128g+128) up
+        const int ldo = p.N / 2;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * ldo + (size_t)nt * (BN / 2);
+#pragma unroll 1
+        for (int g = 0; g < BN / 128; ++g) {
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            float gv[32], uv[32];
+            tmem_ld32(tbase + g * 128 + half * 32, gv);
+            tmem_ld32(tbase + g * 128 + 64 + half * 32, uv);
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(out + g * 64 + half * 32);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                float r[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) r[e] = silu_f(gv[q * 8 + e]) * uv[q * 8 + e];
+                uint4 w;
+                w.x = pack_bf16x2(r[0], r[1]);
+                w.y = pack_bf16x2(r[2], r[3]);
+                w.z = pack_bf16x2(r[4], r[5]);
+                w.w = pack_bf16x2(r[6], r[7]);
+                dst[q] = w;
+              }
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_QKV) {
+        // [q | k | v | gate] columns; 128-wide q/k heads get RMSNorm (1 + w) and RoPE here,
+        // once per element, on the fp32 accumulator (page §四.3 order: norm, then RoPE)
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + (size_t)nt * BN;
+        const int pos = row_ok ? row % p.rows_per_batch : 0;
+        const float* cs = p.cos + (size_t)pos * 64;
+        const float* sn = p.sin + (size_t)pos * 64;
+#pragma unroll 1
+        for (int u = 0; u < BN / 128; ++u) {
+          const int c0 = nt * BN + u * 128;
+          const bool is_q = c0 < p.HD;
+          const bool is_k = !is_q && c0 < p.HD + p.KVD;
+          const uint32_t ub = tbase + u * 128;
+          float r = 1.f;
+          const float* w = is_q ? p.qw : p.kw;
+          if (is_q || is_k) {
+            float ss = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              float v[32];
+              tmem_ld32(ub + c * 32, v);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ss += v[e] * v[e];
+            }
+            r = rsqrtf(ss * (1.f / 128.f) + p.eps);
+          }
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float v[32];
+            tmem_ld32(ub + c * 32, v);
+            if (is_q || is_k) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const int d = c * 32 + e;
+                const float x0 = v[e] * r * (1.f + __ldg(w + d));
+                const float x1 = v[e + 1] * r * (1.f + __ldg(w + d + 1));
+                const float co = __ldg(cs + d / 2), si = __ldg(sn + d / 2);
+                v[e] = x0 * co - x1 * si;
+                v[e + 1] = x1 * co + x0 * si;
+              }
+            }
+            if (row_ok) {
+              uint4* dst = reinterpret_cast<uint4*>(out + u * 128 + c * 32);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint4 w4;
+                w4.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+                w4.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+                w4.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+                w4.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+                dst[q] = w4;
+              }
+            }
+          }
+        }
+      } else {  // EPI_RESID: h[row, col] += gate[b, col] * acc
+        float* hrow = reinterpret_cast<float*>(p.out) + (size_t)row * p.N + (size_t)nt * BN;
+        const int b = row_ok ? row / p.rows_per_batch : 0;
+        const float* grow = p.gate + (size_t)b * p.gate_stride + (size_t)nt * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+          if (row_ok) {
+            float4* hp = reinterpret_cast<float4*>(hrow + c * 32);
+            const float4* gp = reinterpret_cast<const float4*>(grow + c * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 hv = hp[q];
+              const float4 gv = __ldg(gp + q);
+              hv.x += gv.x * v[q * 4 + 0];
+              hv.y += gv.y * v[q * 4 + 1];
+              hv.z += gv.z * v[q * 4 + 2];
+              hv.w += gv.w * v[q * 4 + 3];
+              hp[q] = hv;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (abort_flag) {
+    // give TMA copies that may still be in flight time to land before the CTA exits
+    unsigned long long t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 1000000ull) {
+    }
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// Row-major bf16 matrix (rows, cols) as a 2-D TMA map with a (box_cols x box_rows) box and
+// 128-byte swizzle (box_cols * 2 bytes must be 128).
+int make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_stride_elems,
+                      uint32_t box_cols, uint32_t box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((row_stride_elems * 2) & 15))
+    return set_error(KREA2_ERR_ARG, "TMA operand must be 16-byte aligned with a 16-byte multiple row stride");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return KREA2_OK;
+}
+
+// Row-major bf16 matrix viewed as (batches, rows, cols) with `row_stride_elems` between rows and
+// rows*row_stride between batches; box (box_cols x box_rows x 1), 128-byte swizzle. Rows past
+// `rows` in a batch read as zero.
+int make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t batches,
+                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((row_stride_elems * 2) & 15))
+    return set_error(KREA2_ERR_ARG, "TMA operand must be 16-byte aligned with a 16-byte multiple row stride");
+  cuuint64_t dims[3] = {cols, rows, batches};
+  cuuint64_t strides[2] = {row_stride_elems * 2, row_stride_elems * 2 * rows};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+  return KREA2_OK;
+}
+
+namespace {
+
+template <int BN, int EPI>
+int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN>;
+  static bool attr_done = false;
+  auto kern = gemm_bf16_tcgen05_kernel<BN, EPI>;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
+      return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(gemm) failed");
+    attr_done = true;
+  }
+  CUtensorMap ta, tb;
+  int rc = make_tmap_bf16_2d(&ta, A, p0.K, p0.M, p0.K, BK, BM);
+  if (rc) return rc;
+  rc = make_tmap_bf16_2d(&tb, W, p0.K, p0.N, p0.K, BK, BN);
+  if (rc) return rc;
+  GemmParams p = p0;
+  p.tiles_m = (p.M + BM - 1) / BM;
+  p.tiles_n = p.N / BN;
+  const int total = p.tiles_m * p.tiles_n;
+  const int grid = total < num_sms() ? total : num_sms();
+  kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "gemm launch failed: %s", cudaGetErrorString(e));
+  return KREA2_OK;
+}
+
+// Wave efficiency of a tile count on the SMs (1.0 = every wave full).
+double wave_eff(long tiles, int sms) {
+  long waves = (tiles + sms - 1) / sms;
+  return (double)tiles / (double)(waves * sms);
+}
+
+}  // namespace
+
+KREA2_DEFINE_ERROR_READER(take_device_error_gemm)
+
+int gemm_bf16(int epi, const GemmParams& p, const void* A, const void* W, cudaStream_t stream) {
+  // choose the N tile: 256 unless 128 fills the machine clearly better
+  const int sms = num_sms();
+  const long tm = (p.M + BM - 1) / BM;
+  int bn = 128;
+  if (p.N % 256 == 0) {
+    const double e256 = wave_eff(tm * (p.N / 256), sms);
+    const double e128 = wave_eff(tm * (p.N / 128), sms);
+    bn = (e256 >= 0.8 * e128 || tm * (p.N / 256) >= 4L * sms) ? 256 : 128;
+  }
+  if (bn == 256) {
+    switch (epi) {
+      case EPI_STORE: return launch_gemm_bn<256, EPI_STORE>(p, A, W, stream);
+      case EPI_SWIGLU: return launch_gemm_bn<256, EPI_SWIGLU>(p, A, W, stream);
+      case EPI_QKV: return launch_gemm_bn<256, EPI_QKV>(p, A, W, stream);
+      default: return launch_gemm_bn<256, EPI_RESID>(p, A, W, stream);
+    }
+  }
+  switch (epi) {
+    case EPI_STORE: return launch_gemm_bn<128, EPI_STORE>(p, A, W, stream);
+    case EPI_SWIGLU: return launch_gemm_bn<128, EPI_SWIGLU>(p, A, W, stream);
+    case EPI_QKV: return launch_gemm_bn<128, EPI_QKV>(p, A, W, stream);
+    default: return launch_gemm_bn<128, EPI_RESID>(p, A, W, stream);
+  }
+}
+
+}  // namespace krea2

@@ -1,0 +1,417 @@
+// C ABI entry points (include/krea2.h): argument checks, workspace carving and the launch
+// sequence of the block and the backbone. Every step runs in this library's kernels.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <vector>
+
+#include <cuda_bf16.h>
+
+#include "krea2_internal.h"
+
+namespace krea2 {
+
+static thread_local char g_err[512] = "";
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// [ARCH] §三: sum(axes_dims_rope) == attention_head_dim, else ValueError; plus the limits of
+// this build's kernels.
+int check_dims(const Krea2Dims* d, int dtype) {
+  if (!d) return set_error(KREA2_ERR_ARG, "dims is NULL");
+  if (dtype != KREA2_BF16 && dtype != KREA2_F32) return set_error(KREA2_ERR_ARG, "unknown dtype %d", dtype);
+  if (d->H <= 0 || d->Hkv <= 0 || d->D <= 0 || d->C <= 0 || d->F <= 0)
+    return set_error(KREA2_ERR_ARG, "non-positive model dimension");
+  if (d->C != d->H * d->D) return set_error(KREA2_ERR_ARG, "hidden size C=%d != heads*head_dim=%d", d->C, d->H * d->D);
+  if (d->H % d->Hkv) return set_error(KREA2_ERR_ARG, "heads %d not a multiple of kv heads %d", d->H, d->Hkv);
+  for (int a = 0; a < 3; ++a)
+    if (d->axes[a] < 0 || (d->axes[a] & 1)) return set_error(KREA2_ERR_ARG, "RoPE axis %d has odd size %d", a, d->axes[a]);
+  if (d->axes[0] + d->axes[1] + d->axes[2] != d->D)
+    return set_error(KREA2_ERR_ARG, "sum(axes_dims_rope)=%d != attention_head_dim=%d",
+                     d->axes[0] + d->axes[1] + d->axes[2], d->D);
+  if (!(d->theta > 0.f) || !(d->eps > 0.f)) return set_error(KREA2_ERR_ARG, "theta and eps must be positive");
+  if (d->D != 64 && d->D != 128) return set_error(KREA2_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (d->C % 128 || d->C > 8192) return set_error(KREA2_ERR_UNSUPPORTED, "hidden size must be a multiple of 128, <= 8192");
+  if (d->F % 64) return set_error(KREA2_ERR_UNSUPPORTED, "intermediate size must be a multiple of 64");
+  return KREA2_OK;
+}
+
+int check_model_dims(const Krea2Dims* d) {
+  if (d->n_layers < 0) return set_error(KREA2_ERR_ARG, "n_layers < 0");
+  if (d->in_ch <= 0) return set_error(KREA2_ERR_ARG, "in_ch must be positive");
+  if (d->t_dim <= 0 || d->t_dim % 8 || d->t_dim > d->C)
+    return set_error(KREA2_ERR_UNSUPPORTED, "t_dim must be a positive multiple of 8 and <= C");
+  return KREA2_OK;
+}
+
+int check_shape(int B, int T, int N) {
+  if (B <= 0) return set_error(KREA2_ERR_ARG, "batch must be positive");
+  if (T < 0) return set_error(KREA2_ERR_ARG, "text length must be >= 0");
+  if (N <= 0) return set_error(KREA2_ERR_ARG, "image_seq_len must be >= 1 (every query then has a valid key)");
+  if ((long long)B * (T + N) > (1LL << 30)) return set_error(KREA2_ERR_ARG, "too many tokens");
+  return KREA2_OK;
+}
+
+constexpr size_t ALIGN = 256;
+inline size_t up(size_t x) { return (x + ALIGN - 1) & ~(ALIGN - 1); }
+
+struct Ws {
+  size_t mod, xn, qkvg, attn, u, h, cs, sn, temb, e, tscr, ybuf, total;
+};
+
+Ws ws_layout(const Krea2Dims* d, int B, int T, int N, int dtype) {
+  const size_t es = dtype == KREA2_BF16 ? 2 : 4;
+  const size_t S = (size_t)T + N, M = (size_t)B * S, C = d->C;
+  const size_t QC = 2 * (size_t)d->H * d->D + 2 * (size_t)d->Hkv * d->D;
+  Ws w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += up(bytes);
+    return o;
+  };
+  w.mod = take((size_t)B * 6 * C * 4);
+  w.xn = take(M * C * es);
+  w.qkvg = take(M * QC * es);
+  w.attn = take(M * (size_t)d->H * d->D * es);
+  w.u = take(M * (size_t)d->F * es);
+  w.h = take(M * C * 4);
+  w.cs = take(S * (size_t)(d->D / 2) * 4);
+  w.sn = take(S * (size_t)(d->D / 2) * 4);
+  w.temb = take((size_t)B * 6 * C * 4);
+  w.e = take((size_t)B * C * 4);
+  w.tscr = take((size_t)B * C * 4);
+  w.ybuf = take((size_t)B * N * C * 4);
+  w.total = off;
+  return w;
+}
+
+// Standalone attention on raw projection columns ([ARCH] §四.3): the tensor-core path first
+// writes normalised, rotated q|k into the workspace, then runs the flash-attention core.
+int attention_raw(const AttnParams& p, int dtype, void* ws, cudaStream_t s) {
+  if (dtype == KREA2_BF16 && attention_tc_supported(p.D, p.H, p.Hkv)) {
+    const long long QC = 2LL * p.H * p.D + 2LL * p.Hkv * p.D;
+    int rc = launch_qk_prep(p.qkvg, QC, p.B, p.S, p.H, p.Hkv, p.eps, p.q_norm_w, p.k_norm_w, p.cos, p.sin, ws, s);
+    if (rc) return rc;
+    AttnTcArgs a{};
+    a.B = p.B; a.T = p.T; a.N = p.N; a.H = p.H; a.Hkv = p.Hkv;
+    const long long QK = (long long)(p.H + p.Hkv) * p.D;
+    const __nv_bfloat16* prep = reinterpret_cast<const __nv_bfloat16*>(ws);
+    const __nv_bfloat16* raw = reinterpret_cast<const __nv_bfloat16*>(p.qkvg);
+    a.q = prep; a.q_stride = QK;
+    a.k = prep + (long long)p.H * p.D; a.k_stride = QK;
+    a.v = raw + (long long)(p.H + p.Hkv) * p.D; a.v_stride = QC;
+    a.g = raw + (long long)(p.H + 2 * p.Hkv) * p.D; a.g_stride = QC;
+    a.text_mask = p.text_mask; a.out = p.out;
+    return attention_tc_core(a, s);
+  }
+  return attention_simt(p, dtype == KREA2_BF16, s);
+}
+
+size_t attention_ws_bytes(const Krea2Dims* d, int B, int T, int N, int dtype) {
+  if (dtype == KREA2_BF16 && attention_tc_supported(d->D, d->H, d->Hkv))
+    return (size_t)B * (T + N) * (size_t)(d->H + d->Hkv) * d->D * 2;
+  return 0;
+}
+
+int linear_dispatch(int dtype, int epi, int M, int Nw, int K, const void* A, const void* W, void* out,
+                    const float* gate, int rows_per_batch, long long gate_stride, cudaStream_t s) {
+  if (dtype == KREA2_BF16) {
+    GemmParams p{};
+    p.M = M; p.N = Nw; p.K = K; p.out = out;
+    p.gate = gate; p.rows_per_batch = rows_per_batch; p.gate_stride = gate_stride;
+    return gemm_bf16(epi, p, A, W, s);
+  }
+  SimtGemmParams p{};
+  p.M = M; p.N = Nw; p.K = K; p.out = out;
+  p.gate = gate; p.rows_per_batch = rows_per_batch; p.gate_stride = gate_stride;
+  const int sepi = epi == EPI_STORE ? SEPI_STORE_F32 : epi == EPI_SWIGLU ? SEPI_SWIGLU_F32 : SEPI_RESID;
+  return gemm_simt(sepi, p, A, false, W, false, s);
+}
+
+int check_block_weights(const Krea2BlockWeights* w) {
+  if (!w || !w->w_qkvg || !w->w_out || !w->w_gu || !w->w_down || !w->norm1_w || !w->norm2_w || !w->q_norm_w ||
+      !w->k_norm_w || !w->scale_shift_table)
+    return set_error(KREA2_ERR_ARG, "block weights: NULL pointer");
+  return KREA2_OK;
+}
+
+int check_model_weights(const Krea2ModelWeights* w, int n_layers) {
+  if (!w || !w->img_in_w || !w->img_in_b || !w->t1_w || !w->t1_b || !w->t2_w || !w->t2_b || !w->mod_w ||
+      !w->mod_b || !w->final_norm_w || !w->final_table || !w->final_w || !w->final_b)
+    return set_error(KREA2_ERR_ARG, "model weights: NULL pointer");
+  if (n_layers > 0 && !w->blocks) return set_error(KREA2_ERR_ARG, "model weights: blocks is NULL");
+  for (int l = 0; l < n_layers; ++l) {
+    int rc = check_block_weights(&w->blocks[l]);
+    if (rc) return set_error(rc, "block %d weights: NULL pointer", l);
+  }
+  return KREA2_OK;
+}
+
+// The block's launch sequence ([ARCH] §四.2) on an already validated configuration.
+int block_impl(const Krea2Dims* d, int B, int T, int N, int dtype, float* h, const float* temb,
+               const Krea2BlockWeights* w, const float* cs, const float* sn, const uint8_t* mask, uint8_t* ws,
+               const Ws& L, cudaStream_t s, void* const* ev = nullptr) {
+  auto mark = [&](int i) {
+    if (ev) cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s);
+  };
+  const int S = T + N, M = B * S, C = d->C, HD = d->H * d->D;
+  const int QC = 2 * HD + 2 * d->Hkv * d->D;
+  const bool bf = dtype == KREA2_BF16;
+  float* mod = reinterpret_cast<float*>(ws + L.mod);
+  void* xn = ws + L.xn;
+  void* qkvg = ws + L.qkvg;
+  void* attn = ws + L.attn;
+  void* u = ws + L.u;
+  int rc;
+  mark(0);
+  if ((rc = launch_modulation(temb, w->scale_shift_table, B, C, mod, s))) return rc;
+  mark(1);
+  if ((rc = launch_mod_rmsnorm(h, w->norm1_w, mod, nullptr, 0, B, S, C, d->eps, xn, bf, s))) return rc;
+  if (bf && attention_tc_supported(d->D, d->H, d->Hkv)) {
+    // fused projection with q/k RMSNorm + RoPE in the epilogue, then the tensor-core attention
+    GemmParams gp{};
+    gp.M = M; gp.N = QC; gp.K = C; gp.out = qkvg; gp.rows_per_batch = S;
+    gp.qw = w->q_norm_w; gp.kw = w->k_norm_w; gp.cos = cs; gp.sin = sn;
+    gp.HD = HD; gp.KVD = d->Hkv * d->D; gp.eps = d->eps;
+    mark(2);
+    if ((rc = gemm_bf16(EPI_QKV, gp, xn, w->w_qkvg, s))) return rc;
+    const __nv_bfloat16* base = reinterpret_cast<const __nv_bfloat16*>(qkvg);
+    AttnTcArgs a{};
+    a.B = B; a.T = T; a.N = N; a.H = d->H; a.Hkv = d->Hkv;
+    a.q = base; a.q_stride = QC;
+    a.k = base + HD; a.k_stride = QC;
+    a.v = base + HD + d->Hkv * d->D; a.v_stride = QC;
+    a.g = base + HD + 2 * d->Hkv * d->D; a.g_stride = QC;
+    a.text_mask = mask; a.out = attn;
+    mark(3);
+    if ((rc = attention_tc_core(a, s))) return rc;
+  } else {
+    mark(2);
+    if ((rc = linear_dispatch(dtype, EPI_STORE, M, QC, C, xn, w->w_qkvg, qkvg, nullptr, S, 0, s))) return rc;
+    AttnParams ap{};
+    ap.B = B; ap.T = T; ap.N = N; ap.S = S; ap.H = d->H; ap.Hkv = d->Hkv; ap.D = d->D; ap.eps = d->eps;
+    ap.qkvg = qkvg; ap.q_norm_w = w->q_norm_w; ap.k_norm_w = w->k_norm_w; ap.cos = cs; ap.sin = sn;
+    ap.text_mask = mask; ap.out = attn;
+    mark(3);
+    if ((rc = attention_simt(ap, bf, s))) return rc;
+  }
+  mark(4);
+  if ((rc = linear_dispatch(dtype, EPI_RESID, M, C, HD, attn, w->w_out, h, mod + 2 * C, S, 6LL * C, s))) return rc;
+  mark(5);
+  if ((rc = launch_mod_rmsnorm(h, w->norm2_w, mod, nullptr, 3, B, S, C, d->eps, xn, bf, s))) return rc;
+  mark(6);
+  if ((rc = linear_dispatch(dtype, EPI_SWIGLU, M, 2 * d->F, C, xn, w->w_gu, u, nullptr, S, 0, s))) return rc;
+  mark(7);
+  if ((rc = linear_dispatch(dtype, EPI_RESID, M, C, d->F, u, w->w_down, h, mod + 5 * C, S, 6LL * C, s))) return rc;
+  mark(8);
+  return KREA2_OK;
+}
+
+}  // namespace
+}  // namespace krea2
+
+using namespace krea2;
+
+extern "C" {
+
+const char* krea2_last_error_string(void) { return g_err; }
+
+int krea2_check_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
+  const int ve[2] = {take_device_error_gemm(), take_device_error_attention()};
+  for (int i = 0; i < 2; ++i) {
+    if (ve[i] < 0) return set_error(KREA2_ERR_CUDA, "cannot read the device error word");
+    if (ve[i] > 0)
+      return set_error(KREA2_ERR_TIMEOUT, "a bounded device-side wait expired in the %s kernels (code %d)",
+                       i == 0 ? "GEMM" : "attention", ve[i]);
+  }
+  return KREA2_OK;
+}
+
+size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype) {
+  if (check_dims(dims, dtype) || check_shape(B, T, N)) return 0;
+  return ws_layout(dims, B, T, N, dtype).total;
+}
+
+int krea2_rope_tables(const Krea2Dims* dims, const float* position_ids, int S, float* cos_out, float* sin_out,
+                      void* stream) {
+  int rc = check_dims(dims, KREA2_F32);
+  if (rc) return rc;
+  if (!position_ids || !cos_out || !sin_out) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (S <= 0) return set_error(KREA2_ERR_ARG, "position_ids must have shape (S, 3) with S >= 1");
+  return launch_rope_tables(position_ids, S, dims->axes[0], dims->axes[1], dims->axes[2], dims->theta, cos_out,
+                            sin_out, as_stream(stream));
+}
+
+size_t krea2_attention_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype) {
+  if (check_dims(dims, dtype) || check_shape(B, T, N)) return 0;
+  return attention_ws_bytes(dims, B, T, N, dtype);
+}
+
+int krea2_gqa_attention(const Krea2Dims* dims, int B, int T, int N, int dtype, const void* qkvg,
+                        const float* q_norm_w, const float* k_norm_w, const float* cos, const float* sin,
+                        const uint8_t* text_mask, void* out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_shape(B, T, N))) return rc;
+  if (!qkvg || !q_norm_w || !k_norm_w || !cos || !sin || !out) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  const size_t need = attention_ws_bytes(dims, B, T, N, dtype);
+  if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (ws_bytes < need) return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  AttnParams ap{};
+  ap.B = B; ap.T = T; ap.N = N; ap.S = T + N; ap.H = dims->H; ap.Hkv = dims->Hkv; ap.D = dims->D;
+  ap.eps = dims->eps; ap.qkvg = qkvg; ap.q_norm_w = q_norm_w; ap.k_norm_w = k_norm_w; ap.cos = cos; ap.sin = sin;
+  ap.text_mask = T > 0 ? text_mask : nullptr; ap.out = out;
+  return attention_raw(ap, dtype, workspace, as_stream(stream));
+}
+
+int krea2_modulated_rmsnorm(const Krea2Dims* dims, int B, int S, int dtype, const float* h, const float* norm_w,
+                            const float* temb, const float* table, int chunk, void* out, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc) return rc;
+  if (B <= 0 || S <= 0) return set_error(KREA2_ERR_ARG, "B and S must be positive");
+  if (!h || !norm_w || !temb || !table || !out) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (chunk != 0 && chunk != 3) return set_error(KREA2_ERR_ARG, "chunk must be 0 (norm1) or 3 (norm2)");
+  return launch_mod_rmsnorm(h, norm_w, temb, table, chunk, B, S, dims->C, dims->eps, out, dtype == KREA2_BF16,
+                            as_stream(stream));
+}
+
+int krea2_linear(int dtype, int epilogue, int M, int Nw, int K, const void* A, const void* W, void* out,
+                 const float* gate, int rows_per_batch, long long gate_stride, void* stream) {
+  if (dtype != KREA2_BF16 && dtype != KREA2_F32) return set_error(KREA2_ERR_ARG, "unknown dtype %d", dtype);
+  if (epilogue < EPI_STORE || epilogue > EPI_RESID) return set_error(KREA2_ERR_ARG, "unknown epilogue %d", epilogue);
+  if (M <= 0 || Nw <= 0 || K <= 0) return set_error(KREA2_ERR_ARG, "sizes must be positive");
+  if (!A || !W || !out) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (epilogue == EPI_RESID && (!gate || rows_per_batch <= 0 || gate_stride < 0))
+    return set_error(KREA2_ERR_ARG, "residual epilogue needs gate, rows_per_batch > 0, gate_stride >= 0");
+  if (epilogue == EPI_SWIGLU && Nw % 128) return set_error(KREA2_ERR_ARG, "SwiGLU needs Nw % 128 == 0");
+  if (dtype == KREA2_BF16 && (Nw % 128 || K % 64))
+    return set_error(KREA2_ERR_UNSUPPORTED, "bf16 linear needs Nw %% 128 == 0 and K %% 64 == 0");
+  return linear_dispatch(dtype, epilogue, M, Nw, K, A, W, out, gate, rows_per_batch > 0 ? rows_per_batch : 1,
+                         gate_stride, as_stream(stream));
+}
+
+int krea2_time_embed(const Krea2Dims* dims, int B, int dtype, const float* timestep, const Krea2ModelWeights* w,
+                     float* temb_out, float* e_out, float* scratch, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_model_dims(dims))) return rc;
+  if (B <= 0) return set_error(KREA2_ERR_ARG, "batch must be positive");
+  if (!timestep || !w || !w->t1_w || !w->t1_b || !w->t2_w || !w->t2_b || !w->mod_w || !w->mod_b || !temb_out ||
+      !e_out || !scratch)
+    return set_error(KREA2_ERR_ARG, "NULL pointer");
+  return launch_time_embed(dims, B, dtype == KREA2_BF16, timestep, w, temb_out, e_out, scratch, as_stream(stream));
+}
+
+int krea2_final_layer(const Krea2Dims* dims, int B, int T, int N, int dtype, const float* h, const float* e,
+                      const Krea2ModelWeights* w, void* velocity, float* scratch, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_model_dims(dims)) || (rc = check_shape(B, T, N))) return rc;
+  if (!h || !e || !w || !w->final_norm_w || !w->final_table || !w->final_w || !w->final_b || !velocity || !scratch)
+    return set_error(KREA2_ERR_ARG, "NULL pointer");
+  return launch_final_layer(dims, B, T, N, dtype == KREA2_BF16, h, e, w, scratch, velocity, as_stream(stream));
+}
+
+int krea2_block_forward(const Krea2Dims* dims, int B, int T, int N, int dtype, float* h, const float* temb,
+                        const Krea2BlockWeights* w, const float* cos, const float* sin, const uint8_t* text_mask,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_shape(B, T, N)) || (rc = check_block_weights(w))) return rc;
+  if (!h || !temb || !cos || !sin) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const Ws L = ws_layout(dims, B, T, N, dtype);
+  if (ws_bytes < L.total)
+    return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  return block_impl(dims, B, T, N, dtype, h, temb, w, cos, sin, T > 0 ? text_mask : nullptr,
+                    reinterpret_cast<uint8_t*>(workspace), L, as_stream(stream));
+}
+
+int krea2_block_forward_traced(const Krea2Dims* dims, int B, int T, int N, int dtype, float* h, const float* temb,
+                               const Krea2BlockWeights* w, const float* cos, const float* sin,
+                               const uint8_t* text_mask, void* workspace, size_t ws_bytes, void* const* events,
+                               void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_shape(B, T, N)) || (rc = check_block_weights(w))) return rc;
+  if (!h || !temb || !cos || !sin || !events) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  for (int i = 0; i < 9; ++i)
+    if (!events[i]) return set_error(KREA2_ERR_ARG, "events[%d] is NULL", i);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const Ws L = ws_layout(dims, B, T, N, dtype);
+  if (ws_bytes < L.total)
+    return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  return block_impl(dims, B, T, N, dtype, h, temb, w, cos, sin, T > 0 ? text_mask : nullptr,
+                    reinterpret_cast<uint8_t*>(workspace), L, as_stream(stream), events);
+}
+
+unsigned long long krea2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int krea2_backbone_forward(const Krea2Dims* dims, int B, int T, int N, int dtype, const void* hidden_states,
+                           const void* text_states, const float* position_ids, const uint8_t* text_mask,
+                           const float* timestep, const Krea2ModelWeights* w, void* velocity, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_model_dims(dims)) || (rc = check_shape(B, T, N)) ||
+      (rc = check_model_weights(w, dims->n_layers)))
+    return rc;
+  if (!hidden_states || (T > 0 && !text_states) || !position_ids || !timestep || !velocity)
+    return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const Ws L = ws_layout(dims, B, T, N, dtype);
+  if (ws_bytes < L.total)
+    return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  const bool bf = dtype == KREA2_BF16;
+  const int S = T + N, C = dims->C;
+  float* h = reinterpret_cast<float*>(ws + L.h);
+  float* cs = reinterpret_cast<float*>(ws + L.cs);
+  float* sn = reinterpret_cast<float*>(ws + L.sn);
+  float* temb = reinterpret_cast<float*>(ws + L.temb);
+  float* e = reinterpret_cast<float*>(ws + L.e);
+  if ((rc = launch_rope_tables(position_ids, S, dims->axes[0], dims->axes[1], dims->axes[2], dims->theta, cs, sn, s)))
+    return rc;
+  if ((rc = launch_time_embed(dims, B, bf, timestep, w, temb, e, reinterpret_cast<float*>(ws + L.tscr), s))) return rc;
+  if ((rc = launch_copy_text_rows(text_states, bf, B, T, S, C, h, s))) return rc;
+  SimtGemmParams ip{};
+  ip.M = B * N; ip.N = C; ip.K = dims->in_ch; ip.out = h; ip.bias = w->img_in_b;
+  ip.map_N = N; ip.map_T = T; ip.map_S = S;
+  if ((rc = gemm_simt(SEPI_BIAS_ROWMAP, ip, hidden_states, bf, w->img_in_w, bf, s))) return rc;
+  const uint8_t* mask = T > 0 ? text_mask : nullptr;
+  for (int l = 0; l < dims->n_layers; ++l)
+    if ((rc = block_impl(dims, B, T, N, dtype, h, temb, &w->blocks[l], cs, sn, mask, ws, L, s))) return rc;
+  return launch_final_layer(dims, B, T, N, bf, h, e, w, reinterpret_cast<float*>(ws + L.ybuf), velocity, s);
+}
+
+}  // extern "C"

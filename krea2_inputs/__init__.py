@@ -232,6 +232,8 @@ class Workload:
         return self.B * self.S
 
     def mask(self) -> np.ndarray:
+        if self.T == 0:
+            return np.ones((self.B, 0), dtype=bool)
         return mask_from_lengths(self.T, self.lengths)
 
     def positions(self) -> np.ndarray:

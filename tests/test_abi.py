@@ -1,0 +1,70 @@
+"""The C-ABI library loads without a GPU, exports every entry point of include/krea2.h, and
+rejects bad arguments on the host before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import krea2_inputs as KI
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "krea2.h")
+
+
+@pytest.fixture(scope="module")
+def K2():
+    from flow_matching_stream_b200 import build
+    build.build()
+    import flow_matching_stream_b200 as K2
+    return K2
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(krea2_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_named_entry_points():
+    names = declared_entry_points()
+    for n in ("krea2_rope_tables", "krea2_gqa_attention", "krea2_block_forward", "krea2_backbone_forward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(K2):
+    lib = ctypes.CDLL(os.path.join(ROOT, "flow_matching_stream_b200", "libkrea2.so"))
+    missing = [n for n in declared_entry_points() if not hasattr(lib, n)]
+    assert not missing, missing
+    from flow_matching_stream_b200 import _lib
+    assert sorted(_lib.SIGNATURES) == declared_entry_points()
+
+
+def test_workspace_size_and_dim_checks_on_host(K2):
+    d = K2.dims_struct(KI.FULL)
+    lib = K2.lib()
+    ws = lib.krea2_workspace_size(ctypes.byref(d), 2, 512, 4096, K2.KREA2_BF16)
+    assert ws > 0
+    bad = K2.dims_struct(KI.FULL)
+    bad.axes[2] = 40                      # sum(axes) != head_dim (the pages' ValueError)
+    assert lib.krea2_workspace_size(ctypes.byref(bad), 2, 512, 4096, K2.KREA2_BF16) == 0
+    assert lib.krea2_workspace_size(ctypes.byref(d), 2, 512, 0, K2.KREA2_BF16) == 0   # no image tokens
+    rc = lib.krea2_rope_tables(ctypes.byref(bad), None, 10, None, None, None)
+    assert rc == -1 and b"axes" in lib.krea2_last_error_string()
+    rc = lib.krea2_rope_tables(ctypes.byref(d), None, 10, None, None, None)
+    assert rc == -1 and b"NULL" in lib.krea2_last_error_string()
+    bad2 = K2.dims_struct(KI.FULL)
+    bad2.Hkv = 10
+    assert lib.krea2_block_forward(ctypes.byref(bad2), 1, 8, 8, 0, None, None, None, None, None, None, None, 0,
+                                   None) == -1
+    assert lib.krea2_linear(K2.KREA2_BF16, 0, 128, 100, 64, 1, 1, 1, None, 1, 0, None) == -5   # Nw % 128
+    assert lib.krea2_linear(K2.KREA2_BF16, 7, 128, 128, 64, 1, 1, 1, None, 1, 0, None) == -1   # epilogue
+    assert lib.krea2_attention_workspace_size(ctypes.byref(d), 2, 512, 4096, K2.KREA2_BF16) == \
+        2 * 4608 * (48 + 12) * 128 * 2
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from flow_matching_stream_b200 import _lib
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        _lib.load()

@@ -195,6 +195,24 @@ def cpu_oracle_sample(rows: int = 512) -> dict:
             "kind": "oracle", "sample": o.describe(dt)}
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank number over all ranks (timing is the slowest replica's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, steps: int, flops_per_step: float, ms_max: float) -> float:
+    """Whole-job TFLOP/s of `world` replicas that each ran `steps` steps in at most `ms_max` ms."""
+    return world * steps * flops_per_step / (ms_max / 1e3) / 1e12
+
+
 # ----------------------------------------------------------------------------- native arm
 
 def run_native(args, rank: int, world: int, local_rank: int) -> None:
@@ -212,13 +230,6 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local_rank])
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     warmup = max(args.warmup, 3)
     wl = KI.backbone_1024()
@@ -263,9 +274,9 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     launches = K2.launch_count() - l0
     clk = clocks.stop()
     K2.check_device_error()
-    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
     flops_step = backbone_flops(d, B, T, N, wl.lengths)
-    value = world * args.steps * flops_step / (ms_total / 1e3) / 1e12
+    value = replica_throughput(world, args.steps, flops_step, ms_total)
     ms_step = ms_total / args.steps
 
     # ---- end to end through host buffers: H2D of the step's inputs, forward, D2H of velocity
@@ -288,8 +299,8 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * args.steps * flops_step / (e2e_ms / 1e3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = replica_throughput(world, args.steps, flops_step, e2e_ms)
 
     # ---- per-kernel durations (CUDA events on the launching stream) at the backbone's block shape
     pk = peaks()
@@ -432,6 +443,79 @@ def run_reference(args, rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- single-kernel cases
+
+KERNEL_CASES = ("gate_up", "qkv", "down", "attention", "norm")
+
+
+def run_kernel_case(name: str, steps: int) -> None:
+    """One kernel at the backbone's block shape (M = 4608 tokens), launched `steps` times.
+
+    Small enough for an ncu capture (< 1 GB on the device, inputs larger than L2)."""
+    import torch
+
+    import flow_matching_stream_b200 as K2
+    wl = KI.backbone_1024()
+    d = wl.dims
+    B, T, N, S, M = wl.B, wl.T, wl.N, wl.S, wl.M
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(5)
+    bf = torch.bfloat16
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, device=dev, generator=g) * scale).to(bf)
+
+    if name in ("gate_up", "qkv", "down"):
+        K = d.F if name == "down" else d.C
+        Nw = {"gate_up": 2 * d.F, "qkv": d.qkvg_cols, "down": d.C}[name]
+        A, W = rnd(M, K), rnd(Nw, K, scale=K ** -0.5)
+        if name == "down":
+            out = torch.zeros(M, Nw, device=dev)
+            gate = torch.randn(B, 6 * d.C, device=dev)
+            fn = lambda: K2.linear(K2.KREA2_EPI_RESID, A, W, out, gate=gate.view(-1)[5 * d.C:], rows_per_batch=S,
+                                   gate_stride=6 * d.C)
+        elif name == "gate_up":
+            out = torch.empty(M, d.F, device=dev, dtype=bf)
+            fn = lambda: K2.linear(K2.KREA2_EPI_SWIGLU, A, W, out)
+        else:
+            out = torch.empty(M, Nw, device=dev, dtype=bf)
+            fn = lambda: K2.linear(K2.KREA2_EPI_STORE, A, W, out)
+        flops = 2.0 * M * Nw * K
+    elif name == "attention":
+        x = rnd(M, d.qkvg_cols)
+        qw = torch.randn(d.D, device=dev) * 0.1
+        kw = torch.randn(d.D, device=dev) * 0.1
+        cs = torch.empty(S, d.D // 2, device=dev)
+        sn = torch.empty_like(cs)
+        K2.rope_tables(d, torch.from_numpy(wl.positions()).to(dev), cs, sn)
+        mask = torch.from_numpy(wl.mask().astype(np.uint8)).to(dev)
+        out = torch.empty(M, d.HD, device=dev, dtype=bf)
+        ws = torch.empty(K2.attention_workspace_size(d, B, T, N, bf), dtype=torch.uint8, device=dev)
+        fn = lambda: K2.gqa_attention(d, B, T, N, x, qw, kw, cs, sn, mask, out, ws)
+        flops = 4.0 * d.D * d.H * S * S
+    elif name == "norm":
+        h = torch.randn(M, d.C, device=dev)
+        nw = torch.randn(d.C, device=dev) * 0.1
+        temb = torch.randn(B, 6 * d.C, device=dev)
+        table = torch.randn(6, d.C, device=dev) * 0.1
+        out = torch.empty(M, d.C, device=dev, dtype=bf)
+        fn = lambda: K2.modulated_rmsnorm(d, B, S, h, nw, temb, table, 0, out)
+        flops = 0.0
+    else:
+        raise SystemExit(f"unknown kernel case {name}; choose from {KERNEL_CASES}")
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    K2.check_device_error()
+    ms = e0.elapsed_time(e1) / steps
+    print(json.dumps({"kernel_case": name, "M": M, "ms": ms, "tflops": flops / (ms / 1e3) / 1e12 if flops else None}))
+
+
 def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -439,7 +523,12 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-case", choices=KERNEL_CASES, default=None,
+                    help="run one kernel at the backbone block shape (for profiler captures)")
     args = ap.parse_args()
+    if args.kernel_case:
+        run_kernel_case(args.kernel_case, args.steps)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -20,7 +20,7 @@ from ._lib import KREA2_BF16, KREA2_F32, KREA2_EPI_RESID, KREA2_EPI_STORE, KREA2
 __all__ = [
     "Krea2Error", "lib", "dims_struct", "dtype_code", "workspace_size", "attention_workspace_size",
     "rope_tables", "gqa_attention", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
-    "block_forward", "block_forward_traced", "launch_count", "backbone_forward", "check_device_error", "BlockWeights", "ModelWeights",
+    "block_forward", "block_forward_traced", "BLOCK_STEPS", "launch_count", "backbone_forward", "check_device_error", "BlockWeights", "ModelWeights",
     "interleave_gate_up", "KREA2_BF16", "KREA2_F32", "KREA2_EPI_STORE", "KREA2_EPI_SWIGLU", "KREA2_EPI_RESID",
 ]
 
@@ -165,6 +165,10 @@ def block_forward_traced(dims, B: int, T: int, N: int, h: torch.Tensor, temb: to
     """block_forward recording events[i] before launch i (BLOCK_STEPS order) and events[8] after."""
     if len(events) != 9:
         raise ValueError("need 9 events")
+    st = stream if stream is not None else torch.cuda.current_stream()
+    for e in events:
+        if not e.cuda_event:
+            e.record(st)  # torch creates the CUDA event lazily, on its first record
     arr = (ctypes.c_void_p * 9)(*[e.cuda_event for e in events])
     _want(h, torch.float32, "h")
     _check(lib().krea2_block_forward_traced(ctypes.byref(dims_struct(dims)), B, T, N, bw.dtype_code, _p(h), _p(temb),

@@ -11,6 +11,7 @@ LIB_PATH = os.path.join(HERE, "libkrea2.so")
 KREA2_OK, KREA2_ERR_ARG, KREA2_ERR_WORKSPACE, KREA2_ERR_CUDA, KREA2_ERR_TIMEOUT, KREA2_ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
 KREA2_BF16, KREA2_F32 = 0, 1
 KREA2_EPI_STORE, KREA2_EPI_SWIGLU, KREA2_EPI_RESID = 0, 1, 2
+KREA2_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class Krea2Dims(ctypes.Structure):
@@ -54,6 +55,7 @@ SIGNATURES = {
     "krea2_block_forward_traced": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, _PB, V, V, V, V, c_size_t,
                                            POINTER(c_void_p), V]),
     "krea2_launch_count": (ctypes.c_ulonglong, []),
+    "krea2_gqa_attention_noalloc": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V]),
 }
 
 

@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 OUT = os.path.join(HERE, "libkrea2.so")
 BUILD = os.path.join(ROOT, "_build")
-SOURCES = ["krea2_api.cu", "simt.cu", "gemm_tcgen05.cu", "attention_tc.cu"]
+SOURCES = ["krea2_api.cu", "simt.cu", "gemm_tcgen05.cu", "attention_tc.cu", "attention_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", os.path.join(ROOT, "include")]

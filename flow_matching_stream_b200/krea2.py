@@ -19,7 +19,7 @@ from ._lib import KREA2_BF16, KREA2_F32, KREA2_EPI_RESID, KREA2_EPI_STORE, KREA2
 
 __all__ = [
     "Krea2Error", "lib", "dims_struct", "dtype_code", "workspace_size", "attention_workspace_size",
-    "rope_tables", "gqa_attention", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
+    "rope_tables", "gqa_attention", "gqa_attention_noalloc", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
     "block_forward", "block_forward_traced", "BLOCK_STEPS", "launch_count", "backbone_forward", "check_device_error", "BlockWeights", "ModelWeights",
     "interleave_gate_up", "KREA2_BF16", "KREA2_F32", "KREA2_EPI_STORE", "KREA2_EPI_SWIGLU", "KREA2_EPI_RESID",
 ]
@@ -115,6 +115,18 @@ def gqa_attention(dims, B: int, T: int, N: int, qkvg: torch.Tensor, q_norm_w: to
     _check(lib().krea2_gqa_attention(ctypes.byref(dims_struct(dims)), B, T, N, dt, _p(qkvg), _p(q_norm_w),
                                      _p(k_norm_w), _p(cos), _p(sin), _p(text_mask), _p(out), _p(workspace), ws,
                                      _s(stream)))
+
+
+def gqa_attention_noalloc(dims, B: int, T: int, N: int, qkvg: torch.Tensor, q_norm_w: torch.Tensor,
+                          k_norm_w: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor,
+                          text_mask: Optional[torch.Tensor], out: torch.Tensor, stream=None) -> None:
+    """gqa_attention for callers that cannot allocate: the library's static scratch replaces the workspace."""
+    _want(out, qkvg.dtype, "out")
+    if text_mask is not None:
+        _want(text_mask, torch.uint8, "text_mask")
+    _check(lib().krea2_gqa_attention_noalloc(ctypes.byref(dims_struct(dims)), B, T, N, dtype_code(qkvg.dtype),
+                                             _p(qkvg), _p(q_norm_w), _p(k_norm_w), _p(cos), _p(sin),
+                                             _p(text_mask), _p(out), _s(stream)))
 
 
 def modulated_rmsnorm(dims, B: int, S: int, h: torch.Tensor, norm_w: torch.Tensor, temb: torch.Tensor,

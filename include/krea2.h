@@ -155,6 +155,25 @@ int krea2_gqa_attention(const Krea2Dims* dims, int B, int T, int N, int dtype,
                         const float* cos, const float* sin, const uint8_t* text_mask,
                         void* out, void* workspace, size_t ws_bytes, void* stream);
 
+/* Attention without device allocation. The pages have no counterpart of this entry point:
+ * it exists for callers that cannot hand the library a workspace, such as a plugin interface
+ * that passes only input and output buffers, or a runtime whose allocator owns all device
+ * memory and forbids side allocations while it serves.
+ * Arguments, layouts and results are those of krea2_gqa_attention. The q|k scratch that call
+ * takes from its workspace lives here in a file-scope device array of
+ * KREA2_NOALLOC_SCRATCH_BYTES, resident on every GPU that loads it until the process exits.
+ * Shapes needing more scratch than that (B*(T+N)*(H+Hkv)*D*2 bytes on the tensor-core path;
+ * 4369 tokens at the default 48/12 heads x 128) are rejected with KREA2_ERR_WORKSPACE before
+ * anything runs. The call allocates and frees nothing. The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device current, so it should
+ * come before any stream capture. All calls share the array and it keeps the last call's
+ * contents (nothing in it needs to start at zero), so calls that overlap on the GPU race. */
+#define KREA2_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int krea2_gqa_attention_noalloc(const Krea2Dims* dims, int B, int T, int N, int dtype,
+                                const void* qkvg, const float* q_norm_w, const float* k_norm_w,
+                                const float* cos, const float* sin, const uint8_t* text_mask,
+                                void* out, void* stream);
+
 /* Shared modulation of one block plus its table, then a modulated RMSNorm ([ARCH] §四.2,
  * §四.4): with mod = temb (B, 6C) viewed as (B, 6, C) plus table (6, C),
  *   out[b, s] = (1 + mod[b, chunk]) * rms(h[b, s]) * (1 + norm_w) + mod[b, chunk + 1].

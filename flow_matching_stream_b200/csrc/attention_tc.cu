@@ -6,19 +6,22 @@
 // repeat_interleave order), the text padding mask removes keys, and the merged heads are
 // multiplied by sigmoid(to_gate(x)).
 //
-// Kernel layout (one CTA per (32 query positions, KV head j, batch row b)):
+// Kernel layout (one CTA per (32 query positions, KV head j, batch row b); two CTAs per SM):
 //   * The 128-row MMA tile stacks the 4 query heads of KV head j: row r = 32*hl + p holds head
 //     4j+hl at position p0+p. One K/V tile in shared memory therefore serves all four heads
 //     (K/V are never copied per query head).
-//   * warp 0: TMA producer (Q once; K and V 128-key tiles, 2-stage ring). No cluster multicast.
-//   * warp 1: MMA issuer. S_i = Q K_iᵀ into one of two TMEM score buffers, O += P_{i-1} V_{i-1}
-//     into the TMEM output accumulator (V is the MN-major B operand, P the K-major A operand in
-//     shared memory).
-//   * warps 2..5: softmax, one thread per tile row (TMEM lane): row max from TMEM, lazy
-//     rescaling of O (only when the running max grows by more than 2^8), P = exp2 in bf16 to
-//     shared memory, final 1/l and sigmoid(gate) epilogue.
-//   * Key tiles whose 128 keys are all padded text are skipped entirely; partially padded
-//     tiles and the ragged end of the sequence are masked per key.
+//   * warp 0: TMA producer (Q once; K and V 64-key tiles, 2-stage ring). No cluster multicast.
+//   * warp 1: MMA issuer. S_i = Q K_iᵀ into one of two TMEM score buffers; P_i (bf16, written
+//     back over its own scores) is the TMEM A operand of O += P_i V_i, V being the MN-major B
+//     operand in shared memory.
+//   * warps 2..5: softmax, one thread per tile row (TMEM lane): one TMEM read of the 64 scores,
+//     row max, exp2 into bf16 P in TMEM, then (after P_{i-1} V_{i-1} has landed) lazy
+//     rescaling of O, only when the running max grows by more than 2^8; final 1/l and
+//     sigmoid(gate) epilogue.
+//   * 96 KB of shared memory and 256 TMEM columns per CTA let two CTAs share an SM, so each
+//     SM sub-partition interleaves two independent softmax warps with the MMAs.
+//   * Key tiles whose keys are all padded text are skipped entirely; partially padded tiles and
+//     the ragged end of the sequence are masked per key, full tiles take a mask-free path.
 // q and k arrive already RMS-normalised and rotated (the fused projection's epilogue or the
 // prep kernel below does that once per element); v and gate are raw projection columns.
 #include <cuda.h>
@@ -36,20 +39,20 @@ namespace {
 constexpr int AD = 128;          // head dim
 constexpr int AG = 4;            // query heads per KV head
 constexpr int QPOS = 32;         // query positions per CTA (x4 heads = 128 MMA rows)
-constexpr int KT = 128;          // keys per tile
+constexpr int KT = 64;           // keys per tile
 constexpr int KV_STAGES = 2;
 constexpr int ATT_THREADS = 192;
-constexpr int CHUNK_BYTES = 128 * 128;            // 128 rows x 64 bf16 (128 B) = 16 KB
-constexpr int Q_BYTES = 2 * CHUNK_BYTES;          // 32 KB
-constexpr int KV_TILE_BYTES = 2 * CHUNK_BYTES;    // 32 KB each for K and V
-constexpr int P_BYTES = 2 * CHUNK_BYTES;          // 32 KB
+constexpr int Q_CHUNK = 128 * 128;                // 128 rows x 64 bf16 (128 B) = 16 KB
+constexpr int Q_BYTES = 2 * Q_CHUNK;              // 32 KB
+constexpr int KV_CHUNK = KT * 128;                // 64 rows x 128 B = 8 KB
+constexpr int KV_TILE_BYTES = 2 * KV_CHUNK;       // 16 KB each for K and V
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + Q_BYTES;
 constexpr int OFF_V = OFF_K + KV_STAGES * KV_TILE_BYTES;
-constexpr int OFF_P = OFF_V + KV_STAGES * KV_TILE_BYTES;
-constexpr int ATT_SMEM = OFF_P + P_BYTES + 1024;
-constexpr int MAX_TILES = 512;   // S <= 65536
-constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256,384)
+constexpr int ATT_SMEM = OFF_V + KV_STAGES * KV_TILE_BYTES + 1024;  // + alignment slack
+constexpr int MAX_TILES = 1024;  // S <= 65536
+constexpr uint32_t TMEM_COLS = 256;  // S0 [0,64), S1 [64,128), O [128,256)
+constexpr uint32_t O_COL = 128;
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, KT, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AD, 0, 1);
 
@@ -74,7 +77,7 @@ __device__ __forceinline__ bool key_valid(const AttnCore& p, int b, int t) {
   return true;
 }
 
-__global__ void __launch_bounds__(ATT_THREADS, 1)
+__global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, AttnCore p) {
   extern __shared__ uint8_t smem_raw[];
@@ -150,39 +153,39 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       for (int hl = 0; hl < AG; ++hl)
 #pragma unroll
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(base + OFF_Q + c * CHUNK_BYTES + hl * (QPOS * 128), &tmQ, &q_full,
-                      (j * AG + hl) * AD + c * 64, p0, b);
+          tma_load_3d(base + OFF_Q + c * Q_CHUNK + hl * (QPOS * 128), &tmQ, &q_full, (j * AG + hl) * AD + c * 64,
+                      p0, b);
       for (int i = 0; i < n; ++i) {
         const int st = i % KV_STAGES;
         const uint32_t ph = (i / KV_STAGES) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1, abort)) break;
         const int t0 = tiles[i] * KT;
+        uint8_t* kd = base + OFF_K + st * KV_TILE_BYTES;
+        uint8_t* vd = base + OFF_V + st * KV_TILE_BYTES;
         mbar_arrive_expect_tx(&k_full[st], KV_TILE_BYTES);
-        tma_load_3d(base + OFF_K + st * KV_TILE_BYTES, &tmK, &k_full[st], j * AD, t0, b);
-        tma_load_3d(base + OFF_K + st * KV_TILE_BYTES + CHUNK_BYTES, &tmK, &k_full[st], j * AD + 64, t0, b);
+        tma_load_3d(kd, &tmK, &k_full[st], j * AD, t0, b);
+        tma_load_3d(kd + KV_CHUNK, &tmK, &k_full[st], j * AD + 64, t0, b);
         mbar_arrive_expect_tx(&v_full[st], KV_TILE_BYTES);
-        tma_load_3d(base + OFF_V + st * KV_TILE_BYTES, &tmV, &v_full[st], j * AD, t0, b);
-        tma_load_3d(base + OFF_V + st * KV_TILE_BYTES + CHUNK_BYTES, &tmV, &v_full[st], j * AD + 64, t0, b);
+        tma_load_3d(vd, &tmV, &v_full[st], j * AD, t0, b);
+        tma_load_3d(vd + KV_CHUNK, &tmV, &v_full[st], j * AD + 64, t0, b);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t sq = smem_u32(base + OFF_Q);
-      const uint32_t sp = smem_u32(base + OFF_P);
       bool issued = false;
       auto issue_pv = [&](int i) -> bool {
-        // O += P_i V_i : A = P (K-major over keys), B = V (MN-major: d contiguous per key)
+        // O += P_i V_i : A = P_i in TMEM (bf16 pairs over its scores), B = V (MN-major)
         const int st = i % KV_STAGES;
         if (!mbar_wait(&p_full, i & 1, abort)) return false;
         if (!mbar_wait(&v_full[st], (i / KV_STAGES) & 1, abort)) return false;
         tc_fence_after();
         const uint32_t sv = smem_u32(base + OFF_V + st * KV_TILE_BYTES);
+        const uint32_t pt = tmem + (i & 1) * KT;
 #pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sp + (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sv + kk * 16 * 128, CHUNK_BYTES, 1024);
-          tc_mma_bf16(tmem + 256, ad, bd, IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < KT / 16; ++kk)
+          tc_mma_bf16_ts(tmem + O_COL, pt + kk * 8, smem_desc_sw128(sv + kk * 16 * 128, KV_CHUNK, 1024), IDESC_PV,
+                         (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&pv_done);
         tc_commit(&kv_empty[st]);
         return true;
@@ -193,11 +196,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           if (!mbar_wait(&k_full[st], (i / KV_STAGES) & 1, abort)) break;
           tc_fence_after();
           const uint32_t sk = smem_u32(base + OFF_K + st * KV_TILE_BYTES);
-          const uint32_t d_s = tmem + (i & 1) * 128;
+          const uint32_t d_s = tmem + (i & 1) * KT;
 #pragma unroll
           for (int kk = 0; kk < AD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32;
-            tc_mma_bf16(d_s, smem_desc_sw128(sq + off, 16, 1024), smem_desc_sw128(sk + off, 16, 1024), IDESC_QK,
+            const uint32_t qo = (kk >> 2) * Q_CHUNK + (kk & 3) * 32;
+            const uint32_t ko = (kk >> 2) * KV_CHUNK + (kk & 3) * 32;
+            tc_mma_bf16(d_s, smem_desc_sw128(sq + qo, 16, 1024), smem_desc_sw128(sk + ko, 16, 1024), IDESC_QK,
                         kk > 0 ? 1u : 0u);
           }
           issued = true;
@@ -216,79 +220,66 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   } else {
     // ---- softmax warps: quarter q of the tile = query head 4j+q, rows = 32 positions
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
-    uint8_t* prow = base + OFF_P + row * 128;
     bool ok = true;
     for (int i = 0; i < n && ok; ++i) {
       const int sb = i & 1;
       if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const int t0 = tiles[i] * KT;
-      const bool partial = (t0 < p.T && p.text_mask) || (t0 + KT > p.S);
-      uint32_t vmask[4] = {~0u, ~0u, ~0u, ~0u};
-      if (partial) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) vmask[c] = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + c * 32 + lane));
-      }
-      const uint32_t sbase = tmem + lane_off + sb * 128;
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(sbase + c * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if ((vmask[c] >> e) & 1u) mx = fmaxf(mx, v[e]);
-      }
-      const float mnew = fmaxf(m, mx * sl2);
-      if (i >= 1 && !mbar_wait(&pv_done, (i - 1) & 1, abort)) { ok = false; break; }
-      tc_fence_after();
-      const bool grow = mnew > m + 8.0f;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float alpha = grow ? ex2(m - mnew) : 1.f;  // m = -inf on the first tile -> 0
-        if (i >= 1) {
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(tmem + lane_off + 256 + c * 32, o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tmem + lane_off + 256 + c * 32, o);
-          }
-          tmem_wait_st();
-        }
-        if (grow) {
-          l *= alpha;
-          m = mnew;
-        }
-      }
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(sbase + c * 32, v);
-        float pr[32];
+      const uint32_t sbase = tmem + lane_off + sb * KT;
+      float v[KT];
+      tmem_ld32(sbase, v);
+      tmem_ld32(sbase + 32, v + 32);
+      if ((t0 < p.T && p.text_mask) || (t0 + KT > p.S)) {  // warp-uniform: only partial tiles mask
+        const uint32_t vm0 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + lane));
+        const uint32_t vm1 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + 32 + lane));
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          pr[e] = ((vmask[c] >> e) & 1u) ? ex2(v[e] * sl2 - m) : 0.f;
-          l += pr[e];
-        }
-        // keys 32c..32c+31 -> chunk c/2, 16-byte granules 4*(c%2)..+3, 128-byte swizzle
-        uint8_t* chunk = prow + (c >> 1) * CHUNK_BYTES;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int gran = (c & 1) * 4 + g;
-          uint4 w;
-          w.x = pack_bf16x2(pr[g * 8 + 0], pr[g * 8 + 1]);
-          w.y = pack_bf16x2(pr[g * 8 + 2], pr[g * 8 + 3]);
-          w.z = pack_bf16x2(pr[g * 8 + 4], pr[g * 8 + 5]);
-          w.w = pack_bf16x2(pr[g * 8 + 6], pr[g * 8 + 7]);
-          *reinterpret_cast<uint4*>(chunk + ((gran ^ (row & 7)) << 4)) = w;
+          if (!((vm0 >> e) & 1u)) v[e] = -INFINITY;
+          if (!((vm1 >> e) & 1u)) v[32 + e] = -INFINITY;
         }
       }
-      fence_proxy_async_smem();
+      float mx = v[0];
+#pragma unroll
+      for (int e = 1; e < KT; ++e) mx = fmaxf(mx, v[e]);
+      const float mnew = fmaxf(m, mx * sl2);
+      const bool grow = mnew > m + 8.0f;  // m = -inf on the first tile
+      float alpha = 1.f;
+      if (grow) {
+        alpha = ex2(m - mnew);  // 0 on the first tile
+        m = mnew;
+      }
+      const bool any_grow = __any_sync(0xffffffffu, grow);
+      uint32_t pk[KT / 2];
+      float rs = 0.f;
+#pragma unroll
+      for (int e = 0; e < KT / 2; ++e) {
+        const float a = ex2(fmaf(v[2 * e], sl2, -m));
+        const float c = ex2(fmaf(v[2 * e + 1], sl2, -m));
+        rs += a + c;
+        pk[e] = pack_bf16x2(a, c);
+      }
+      l = l * alpha + rs;
+      tmem_st32(sbase, reinterpret_cast<const float*>(pk));  // P_i over the first 32 score columns
+      if (i >= 1) {
+        // O must hold P_{i-1} V_{i-1} before it is rescaled (also keeps the phase count exact)
+        if (!mbar_wait(&pv_done, (i - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        if (any_grow) {
+#pragma unroll 1
+          for (int c = 0; c < AD / 32; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_off + O_COL + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tmem + lane_off + O_COL + c * 32, o);
+          }
+        }
+      }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full);
     }
@@ -300,9 +291,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const long grow_idx = (long)b * p.S + pos;
       const float inv_l = 1.f / l;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < AD / 32; ++c) {
         float o[32];
-        tmem_ld32(tmem + lane_off + 256 + c * 32, o);
+        tmem_ld32(tmem + lane_off + O_COL + c * 32, o);
         if (row_ok) {
           const uint4* gp = reinterpret_cast<const uint4*>(p.gate + grow_idx * p.g_stride + h * AD + c * 32);
           uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD + c * 32);
@@ -380,7 +371,9 @@ int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(attn_gqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(attn_gqa_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(attention) failed");
     attr_done = true;
   }

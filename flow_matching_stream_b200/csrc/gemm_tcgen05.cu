@@ -15,8 +15,8 @@
 //   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane), reads 32 columns
 //               at a time with tcgen05.ld and applies the fused epilogue, while the MMA warp
 //               already accumulates the next tile into the other TMEM buffer.
-// Tiles are visited in groups of GROUP_M row-tiles so that concurrently running CTAs share
-// W and A tiles through L2.
+// Tiles are visited in groups of row tiles (sized so the group's A tiles stay in L2) so that
+// concurrently running CTAs share W and A tiles through L2.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -29,7 +29,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int GROUP_M = 16;
+// Row tiles per raster group: as many as keep the group's A tiles (128 x K bf16 each) within
+// about 48 MB of L2, so W streams from HBM about once per group pass.
+constexpr size_t GROUP_A_BYTES = 48ull << 20;
 constexpr int GEMM_THREADS = 192;
 
 template <int BN>
@@ -44,12 +46,12 @@ struct GemmCfg {
 };
 
 struct TileMap {
-  int tiles_m, tiles_n;
+  int tiles_m, tiles_n, group_m;
   __device__ __forceinline__ void map(int t, int& mt, int& nt) const {
-    int per_group = GROUP_M * tiles_n;
+    int per_group = group_m * tiles_n;
     int g = t / per_group;
-    int first_m = g * GROUP_M;
-    int gsize = min(tiles_m - first_m, GROUP_M);
+    int first_m = g * group_m;
+    int gsize = min(tiles_m - first_m, group_m);
     int local = t - g * per_group;
     mt = first_m + local % gsize;
     nt = local / gsize;
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const uint32_t tmem_base = tmem_slot;
   volatile int* abort = &abort_flag;
 
-  const TileMap tm{p.tiles_m, p.tiles_n};
+  const TileMap tm{p.tiles_m, p.tiles_n, p.group_m};
   const int total = p.tiles_m * p.tiles_n;
   const int nk = p.K / BK;
 
@@ -400,6 +402,12 @@ int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStrea
   GemmParams p = p0;
   p.tiles_m = (p.M + BM - 1) / BM;
   p.tiles_n = p.N / BN;
+  {
+    const size_t per_tile = (size_t)BM * p.K * 2;
+    int g = (int)(GROUP_A_BYTES / per_tile);
+    g = g < 8 ? 8 : g;
+    p.group_m = g < p.tiles_m ? g : p.tiles_m;
+  }
   const int total = p.tiles_m * p.tiles_n;
   const int grid = total < num_sms() ? total : num_sms();
   kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);

@@ -34,6 +34,7 @@ struct GemmParams {
   int HD, KVD;
   float eps;
   int tiles_m, tiles_n;     // filled by the launcher
+  int group_m;              // row tiles per raster group (filled by the launcher)
 };
 
 // tcgen05 bf16 GEMM (gemm_tcgen05.cu). Requires N % 128 == 0, K % 64 == 0.

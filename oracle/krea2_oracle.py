@@ -337,3 +337,40 @@ def backbone_forward(hidden: np.ndarray, text: np.ndarray, pos: np.ndarray,
     for layer in range(n_layers):
         x = block_forward(x, temb, block_w(layer), cos, sin, kv, H, Hkv, D, eps, dtype=dtype)
     return final_layer(x[:, T:], e, mw, eps, dtype)
+
+
+# ----------------------------------------------------------------------------- sampler (Euler + CFG)
+
+def shift_mu(image_seq_len: int, base_seq_len: int = 256, max_seq_len: int = 6400,
+             base_shift: float = 0.5, max_shift: float = 1.15) -> float:
+    """Resolution-aware shift parameter ([PIPE] scheduler: use_dynamic_shifting with base_shift 0.5,
+    max_shift 1.15, base_image_seq_len 256, max_image_seq_len 6400; `mu` is computed from the
+    image resolution unless the checkpoint is distilled, where mu = 1.15).
+    READING: mu is the straight line through (256, 0.5) and (6400, 1.15) in image_seq_len."""
+    slope = (max_shift - base_shift) / (max_seq_len - base_seq_len)
+    return base_shift + slope * (image_seq_len - base_seq_len)
+
+
+def shifted_sigmas(steps: int, mu: float) -> np.ndarray:
+    """Sigma schedule ([PIPE] __call__: default grid linspace(1, 1/N, N); the scheduler applies the
+    exponential time shift). READING: sigma' = e^mu / (e^mu + (1/sigma - 1)), followed by the
+    terminal sigma 0. Returns steps + 1 values in fp64."""
+    s = np.linspace(1.0, 1.0 / steps, steps)
+    em = math.exp(mu)
+    shifted = em / (em + (1.0 / s - 1.0))
+    return np.concatenate([shifted, [0.0]])
+
+
+def cfg_combine(cond: np.ndarray, uncond: Optional[np.ndarray], guidance: float) -> np.ndarray:
+    """Krea 2 guidance convention ([PIPE] guidance_scale): v = cond + g * (cond - uncond), used
+    whenever g > 0; g = 0 returns cond."""
+    if guidance <= 0 or uncond is None:
+        return cond
+    return cond + guidance * (cond - uncond)
+
+
+def euler_step(x: np.ndarray, v: np.ndarray, sigma: float, sigma_next: float) -> np.ndarray:
+    """Flow-matching Euler update of FlowMatchEulerDiscreteScheduler ([PIPE] scheduler):
+    x <- x + (sigma_next - sigma) * v. The model sees timestep = sigma (t / num_train_timesteps,
+    [ARCH] §五)."""
+    return x + (sigma_next - sigma) * v

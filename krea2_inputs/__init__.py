@@ -145,6 +145,51 @@ def model_weights(d: Dims, seed: int = SEED_WEIGHTS) -> Dict[str, np.ndarray]:
     return out
 
 
+@dataclass(frozen=True)
+class TextDims:
+    """Text-fusion hyper-parameters ([API] text_hidden_dim 2560, num_text_layers 12,
+    text_num_attention_heads / text_num_key_value_heads 20, text_intermediate_size 6912,
+    num_layerwise_text_blocks 2, num_refiner_text_blocks 2); C is the backbone hidden size."""
+
+    Dt: int = 2560
+    L: int = 12
+    H: int = 20
+    Hkv: int = 20
+    D: int = 128
+    F: int = 6912
+    n_layerwise: int = 2
+    n_refiner: int = 2
+    C: int = 6144
+    eps: float = 1e-5
+
+    def block_dims(self) -> Dims:
+        # a fusion block has the shapes of a backbone block of hidden size Dt (no RoPE is applied)
+        return Dims(C=self.Dt, H=self.H, Hkv=self.Hkv, D=self.D, F=self.F, axes=(self.D // 4, 3 * self.D // 8,
+                                                                                  3 * self.D // 8), eps=self.eps)
+
+
+FULL_TEXT = TextDims()
+TINY_TEXT = TextDims(Dt=128, L=3, H=2, Hkv=2, D=64, F=256, n_layerwise=1, n_refiner=1, C=256)
+
+
+def text_fusion_weights(td: TextDims, seed: int = SEED_WEIGHTS) -> Dict[str, object]:
+    """Layerwise and refiner block weights, the layer-axis projection (L,) and txt_in (C, Dt) + bias."""
+    bd = td.block_dims()
+    layerwise = [block_weights(bd, 20_000 + i, seed) for i in range(td.n_layerwise)]
+    refiner = [block_weights(bd, 21_000 + i, seed) for i in range(td.n_refiner)]
+    for w in layerwise + refiner:
+        del w["table"]
+    return {"layerwise": layerwise, "refiner": refiner,
+            "layer_w": _normal(seed, (22_000, 0), (td.L,), td.L ** -0.5),
+            "txt_in_w": _normal(seed, (22_000, 1), (td.C, td.Dt), td.Dt ** -0.5),
+            "txt_in_b": _normal(seed, (22_000, 2), (td.C,), 0.1)}
+
+
+def encoder_hidden_states(td: TextDims, B: int, T: int, seed: int = SEED_ACTIVATIONS, key: int = 0) -> np.ndarray:
+    """Stacked text-encoder hidden states (B, T, L, Dt) ~ N(0, 1)."""
+    return _normal(seed, (key, 5), (B, T, td.L, td.Dt), 1.0)
+
+
 def residual(d: Dims, B: int, S: int, seed: int = SEED_ACTIVATIONS, key: int = 0) -> np.ndarray:
     """Residual stream h (B, S, C) ~ N(0, 1)."""
     return _normal(seed, (key, 0), (B, S, d.C), 1.0)

@@ -374,3 +374,77 @@ def euler_step(x: np.ndarray, v: np.ndarray, sigma: float, sigma_next: float) ->
     x <- x + (sigma_next - sigma) * v. The model sees timestep = sigma (t / num_train_timesteps,
     [ARCH] §五)."""
     return x + (sigma_next - sigma) * v
+
+
+def sample(latents: np.ndarray, text_cond: np.ndarray, text_uncond: Optional[np.ndarray],
+           mask_cond: Optional[np.ndarray], mask_uncond: Optional[np.ndarray], pos: np.ndarray,
+           sigmas: Sequence[float], guidance: float, mw: Dict[str, np.ndarray],
+           block_w: Callable[[int], Dict[str, np.ndarray]], n_layers: int, H: int, Hkv: int, D: int,
+           axes: Sequence[int], theta: float, eps: float, t_dim: int, dtype=np.float64) -> np.ndarray:
+    """Sampling loop of [PIPE] __call__ for one image: at each sigma the backbone predicts the
+    velocity for the conditional prompt (and, when guidance > 0, for the unconditional one, as
+    a separate forward), the two are combined with cfg_combine and euler_step moves the latents
+    to the next sigma. latents (N, in_ch); text_* (T, C); masks (T) or None. Returns (N, in_ch)."""
+    x = latents.astype(dtype)
+    for i in range(len(sigmas) - 1):
+        t = np.array([sigmas[i]], dtype=np.float64)
+
+        def velocity(text, mask):
+            m = None if mask is None else mask[None]
+            return backbone_forward(x[None], text[None], pos, m, t, mw, block_w, n_layers, H, Hkv, D, axes,
+                                    theta, eps, t_dim, dtype)[0]
+        vc = velocity(text_cond, mask_cond)
+        vu = velocity(text_uncond, mask_uncond) if guidance > 0 else None
+        x = euler_step(x, cfg_combine(vc, vu, guidance), sigmas[i], sigmas[i + 1])
+    return x
+
+
+# ----------------------------------------------------------------------------- text fusion
+
+def text_fusion_block(x: np.ndarray, w: Dict[str, np.ndarray], key_valid: np.ndarray, H: int, Hkv: int,
+                      D: int, eps: float, dtype=np.float64) -> np.ndarray:
+    """Krea2TextFusionBlock ([ARCH] §四.1): a pre-norm block with no RoPE and no time modulation.
+
+    READING: apart from those two, the same structure as Krea2TransformerBlock:
+    x + attn(norm1(x)), then + SwiGLU(norm2(x)), with q/k RMSNorm and the sigmoid-gated
+    attention of §四.3 (text heads text_num_attention_heads / text_num_key_value_heads). Written
+    as block_forward with a modulation of (scale 0, shift 0, gate 1) twice and a zero rotation,
+    which are exact identities. x (B, S, Dt); key_valid (B, S). Returns (B, S, Dt)."""
+    B, S, C = x.shape
+    unit = np.zeros((6, C))
+    unit[2] = 1.0
+    unit[5] = 1.0
+    wu = dict(w)
+    wu["table"] = unit
+    ang0 = np.zeros((S, D // 2))
+    return block_forward(x, np.zeros((B, 6 * C)), wu, np.cos(ang0), np.sin(ang0), key_valid, H, Hkv, D, eps,
+                         dtype=dtype)
+
+
+def text_fusion(ehs: np.ndarray, text_mask: Optional[np.ndarray], layerwise: Sequence[Dict[str, np.ndarray]],
+                layer_w: np.ndarray, refiner: Sequence[Dict[str, np.ndarray]], H: int, Hkv: int, D: int,
+                eps: float, dtype=np.float64) -> np.ndarray:
+    """Krea2TextFusion ([ARCH] §四.1; sizes from [API] text_* parameters).
+
+    ehs (B, T, L, Dt): L stacked encoder layers per token. Three steps, in the page's order:
+    1. layerwise: each token's (L, Dt) stack is its own sequence through the layerwise blocks
+       (no mask: every layer is valid);
+    2. projection: Linear(L, 1, bias=False) over the layer axis, layer_w (L,);
+    3. refiner: the (B, T, Dt) token sequence through the refiner blocks with the text mask.
+    Returns (B, T, Dt)."""
+    B, T, L, Dt = ehs.shape
+    x = ehs.astype(dtype).reshape(B * T, L, Dt)
+    all_valid = np.ones((B * T, L), dtype=bool)
+    for w in layerwise:
+        x = text_fusion_block(x, w, all_valid, H, Hkv, D, eps, dtype)
+    x = np.einsum("nld,l->nd", x, layer_w.astype(dtype)).reshape(B, T, Dt)
+    kv = np.ones((B, T), dtype=bool) if text_mask is None else np.asarray(text_mask, dtype=bool)
+    for w in refiner:
+        x = text_fusion_block(x, w, kv, H, Hkv, D, eps, dtype)
+    return x
+
+
+def txt_in(x: np.ndarray, w: np.ndarray, b: np.ndarray, dtype=np.float64) -> np.ndarray:
+    """Krea2TextProjection ([ARCH] §四 module list: txt_in(text_hidden_dim -> hidden_size)).
+    READING: its internals are not given; a plain Linear(Dt, C) with bias."""
+    return x.astype(dtype) @ w.astype(dtype).T + b.astype(dtype)

@@ -317,6 +317,9 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     cfg = KI.block_1024_cfg()
     cfg_res = time_block(K2, torch, cfg, dev, args.steps, warmup, pk)
 
+    sampler = time_sampler(K2, torch, d, mw, dev)
+    text = time_text_fusion(K2, torch, dev, args.steps)
+
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -328,7 +331,8 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "flops_per_step": flops_step},
         "backbone_ms_per_step": ms_step,
-        "schedule_ms_forward_only": {"8_step": 8 * ms_step, "28_step": 28 * ms_step},
+        "sampler_1024sq": sampler,
+        "text_fusion_once_per_prompt": text,
         "pct_of_tensor_peak": {"burst": value / world / pk["bf16_tflops"],
                                "sustained": value / world / pk["bf16_tflops_sustained"]},
         "block_1024sq_cfg": cfg_res,
@@ -347,6 +351,99 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def time_sampler(K2, torch, d, mw, dev) -> dict:
+    """The device sampling loop (krea2_sample) at 1024^2 for both presets of the pages: 8 steps
+    without guidance at mu = 1.15 (distilled) and 28 steps with guidance 4.5 at the resolution mu
+    (one batch-2 [cond, uncond] forward per step). Timed eagerly and as a CUDA graph replay."""
+    T, gh, gw = 512, 64, 64
+    N = gh * gw
+    g = torch.Generator(device=dev).manual_seed(9)
+    text_c = torch.randn(T, d.C, device=dev, generator=g).to(torch.bfloat16)
+    text_u = torch.randn(T, d.C, device=dev, generator=g).to(torch.bfloat16)
+    mask_c = torch.ones(T, dtype=torch.uint8, device=dev)
+    mask_u = torch.zeros(T, dtype=torch.uint8, device=dev)
+    mask_u[:8] = 1  # empty negative prompt: a handful of valid tokens
+    pos = torch.from_numpy(KI.position_ids(T, gh, gw)).to(dev)
+    lat0 = torch.randn(N, d.in_ch, device=dev, generator=g)
+    out = {}
+    for name, steps, guidance, mu in (("8_step_distilled", 8, 0.0, 1.15),
+                                      ("28_step_cfg_4.5", 28, 4.5, K2.shift_mu(N))):
+        sig = K2.sigma_schedule(steps, mu)
+        ws = torch.empty(K2.sample_workspace_size(d, T, N, torch.bfloat16, guidance > 0), dtype=torch.uint8,
+                         device=dev)
+        lat = lat0.clone()
+
+        def run():
+            lat.copy_(lat0)
+            K2.sample(d, T, N, lat, text_c, text_u, mask_c, mask_u, pos, sig, guidance, mw, ws)
+
+        run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        run()
+        e1.record()
+        torch.cuda.synchronize()
+        eager = e0.elapsed_time(e1)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            run()
+        torch.cuda.synchronize()
+        e0.record()
+        graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        K2.check_device_error()
+        replay = e0.elapsed_time(e1)
+        finite = bool(torch.isfinite(lat).all().item())
+        del graph
+        out[name] = {"steps": steps, "guidance": guidance, "mu": mu, "eager_s": eager / 1e3,
+                     "graph_replay_s": replay / 1e3, "ms_per_sampler_step": replay / steps,
+                     "forwards_per_step": 2 if guidance > 0 else 1, "finite": finite}
+    return out
+
+
+def time_text_fusion(K2, torch, dev, steps: int) -> dict:
+    """Text conditioning once per prompt at the pages' sizes: a [cond, uncond] batch of 512 tokens
+    x 12 stacked layers x 2560, 2 layerwise + 2 refiner blocks, txt_in to 6144."""
+    td = KI.FULL_TEXT
+    B, T = 2, 512
+    g = torch.Generator(device=dev).manual_seed(13)
+    bd = td.block_dims()
+    rnd = lambda *sh, sc=1.0: (torch.randn(*sh, device=dev, generator=g) * sc)
+
+    def block():
+        C, HD, KVD, F, D = bd.C, bd.HD, bd.KVD, bd.F, bd.D
+        return {"wq": rnd(HD, C, sc=C ** -0.5), "wk": rnd(KVD, C, sc=C ** -0.5), "wv": rnd(KVD, C, sc=C ** -0.5),
+                "wg": rnd(HD, C, sc=C ** -0.5), "wo": rnd(C, HD, sc=HD ** -0.5), "w_gate": rnd(F, C, sc=C ** -0.5),
+                "w_up": rnd(F, C, sc=C ** -0.5), "w_down": rnd(C, F, sc=F ** -0.5), "norm1_w": rnd(C, sc=0.1),
+                "norm2_w": rnd(C, sc=0.1), "q_norm_w": rnd(D, sc=0.1), "k_norm_w": rnd(D, sc=0.1)}
+    tw = K2.TextWeights({"layerwise": [block() for _ in range(td.n_layerwise)],
+                         "refiner": [block() for _ in range(td.n_refiner)], "layer_w": rnd(td.L, sc=td.L ** -0.5),
+                         "txt_in_w": rnd(td.C, td.Dt, sc=td.Dt ** -0.5), "txt_in_b": rnd(td.C, sc=0.1)},
+                        torch.bfloat16, dev)
+    ehs = rnd(B, T, td.L, td.Dt).to(torch.bfloat16)
+    mask = torch.ones(B, T, dtype=torch.uint8, device=dev)
+    mask[1, 8:] = 0
+    out = torch.empty(B, T, td.C, device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(K2.text_fusion_workspace_size(td, B, T, torch.bfloat16), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        K2.text_fusion(td, B, T, ehs, mask, tw, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        K2.text_fusion(td, B, T, ehs, mask, tw, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    K2.check_device_error()
+    ms = e0.elapsed_time(e1) / steps
+    # GEMM FLOPs of the four fusion blocks (B*T*L rows for the layerwise ones) plus txt_in
+    per_row = 2 * bd.C * (bd.qkvg_cols + bd.HD + 2 * bd.F + bd.F)
+    fl = per_row * (td.n_layerwise * B * T * td.L + td.n_refiner * B * T) + 2 * B * T * td.Dt * td.C
+    return {"workload": "text_fusion_2x512x12x2560", "ms": ms, "gemm_tflops": fl / (ms / 1e3) / 1e12}
 
 
 def traced_block_kernels(K2, torch, d, B, T, N, lengths, bw, dev, reps: int) -> dict:

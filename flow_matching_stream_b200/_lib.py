@@ -33,7 +33,19 @@ class Krea2ModelWeights(ctypes.Structure):
                 ("final_b", c_void_p), ("blocks", POINTER(Krea2BlockWeights))]
 
 
+class Krea2TextDims(ctypes.Structure):
+    _fields_ = [("Dt", c_int), ("L", c_int), ("H", c_int), ("Hkv", c_int), ("D", c_int), ("F", c_int),
+                ("n_layerwise", c_int), ("n_refiner", c_int), ("C", c_int), ("eps", c_float)]
+
+
+class Krea2TextWeights(ctypes.Structure):
+    _fields_ = [("layerwise", POINTER(Krea2BlockWeights)), ("refiner", POINTER(Krea2BlockWeights)),
+                ("layer_w", c_void_p), ("txt_in_w", c_void_p), ("txt_in_b", c_void_p)]
+
+
 _PD = POINTER(Krea2Dims)
+_PTD = POINTER(Krea2TextDims)
+_PTW = POINTER(Krea2TextWeights)
 _PB = POINTER(Krea2BlockWeights)
 _PM = POINTER(Krea2ModelWeights)
 V = c_void_p
@@ -49,12 +61,22 @@ SIGNATURES = {
     "krea2_modulated_rmsnorm": (c_int, [_PD, c_int, c_int, c_int, V, V, V, V, c_int, V, V]),
     "krea2_linear": (c_int, [c_int, c_int, c_int, c_int, c_int, V, V, V, V, c_int, c_longlong, V]),
     "krea2_time_embed": (c_int, [_PD, c_int, c_int, V, _PM, V, V, V, V]),
-    "krea2_final_layer": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, _PM, V, V, V]),
+    "krea2_final_layer": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, _PM, V, V]),
     "krea2_block_forward": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, _PB, V, V, V, V, c_size_t, V]),
     "krea2_backbone_forward": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, _PM, V, V, c_size_t, V]),
     "krea2_block_forward_traced": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, _PB, V, V, V, V, c_size_t,
                                            POINTER(c_void_p), V]),
     "krea2_launch_count": (ctypes.c_ulonglong, []),
+    "krea2_shift_mu": (ctypes.c_double, [c_int]),
+    "krea2_sigma_schedule": (c_int, [c_int, ctypes.c_double, V]),
+    "krea2_euler_cfg_step": (c_int, [c_int, c_longlong, V, V, V, c_float, c_float, c_float, V, c_int, V, V]),
+    "krea2_sample_workspace_size": (c_size_t, [_PD, c_int, c_int, c_int, c_int]),
+    "krea2_sample": (c_int, [_PD, c_int, c_int, c_int, V, V, V, V, V, V, V, c_int, c_float, _PM, V, c_size_t, V]),
+    "krea2_text_fusion_workspace_size": (c_size_t, [_PTD, c_int, c_int, c_int]),
+    "krea2_text_fusion": (c_int, [_PTD, c_int, c_int, c_int, V, V, _PTW, V, V, c_size_t, V]),
+    "krea2_block_causal_key_end": (c_int, [V, c_int, V]),
+    "krea2_gqa_attention_block_causal": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V, V,
+                                                 c_size_t, V]),
     "krea2_gqa_attention_noalloc": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V]),
 }
 

@@ -6,10 +6,10 @@
 // repeat_interleave order), the text padding mask removes keys, and the merged heads are
 // multiplied by sigmoid(to_gate(x)).
 //
-// Kernel layout (one CTA per (32 query positions, KV head j, batch row b); two CTAs per SM):
-//   * The 128-row MMA tile stacks the 4 query heads of KV head j: row r = 32*hl + p holds head
-//     4j+hl at position p0+p. One K/V tile in shared memory therefore serves all four heads
-//     (K/V are never copied per query head).
+// Kernel layout (one CTA per (128/G query positions, KV head j, batch row b); two CTAs per SM):
+//   * The 128-row MMA tile stacks the G query heads of KV head j (G = 4 in the Krea 2 block):
+//     row r = QPOS*hl + p holds head G*j+hl at position p0+p, QPOS = 128/G. One K/V tile in
+//     shared memory therefore serves all G heads (K/V are never copied per query head).
 //   * warp 0: TMA producer (Q once; K and V 64-key tiles, 2-stage ring). No cluster multicast.
 //   * warp 1: MMA issuer. S_i = Q K_iᵀ into one of two TMEM score buffers; P_i (bf16, written
 //     back over its own scores) is the TMEM A operand of O += P_i V_i, V being the MN-major B
@@ -37,8 +37,6 @@ int make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
 namespace {
 
 constexpr int AD = 128;          // head dim
-constexpr int AG = 4;            // query heads per KV head
-constexpr int QPOS = 32;         // query positions per CTA (x4 heads = 128 MMA rows)
 constexpr int KT = 64;           // keys per tile
 constexpr int KV_STAGES = 2;
 constexpr int ATT_THREADS = 192;
@@ -63,6 +61,7 @@ struct AttnCore {
   long long g_stride;
   __nv_bfloat16* out;         // (B*S, HD)
   float scale_log2;
+  const int* key_end;         // PREFIX: query q reads keys [0, key_end[q]) only (same for all batch rows)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -71,12 +70,57 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Paired fp32 ops of sm_100: two lanes of work per instruction.
+__device__ __forceinline__ unsigned long long f2u(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void u2f(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long fadd2(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// exp2 of (v * sl2 - m) for 64 scores, packed to bf16 pairs; returns the row sum of the fp32 values.
+__device__ __forceinline__ float exp_tile(const float* v, float sl2, float m, uint32_t* pk) {
+  const unsigned long long s2 = f2u(sl2, sl2), nm2 = f2u(-m, -m);
+  unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    float x0, x1;
+    u2f(ffma2(f2u(v[2 * e], v[2 * e + 1]), s2, nm2), x0, x1);
+    const float a = ex2(x0), c = ex2(x1);
+    pk[e] = pack_bf16x2(a, c);
+    acc[e & 3] = fadd2(acc[e & 3], f2u(a, c));
+  }
+  float t[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) u2f(acc[k], t[2 * k], t[2 * k + 1]);
+  return ((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7]));
+}
+
 __device__ __forceinline__ bool key_valid(const AttnCore& p, int b, int t) {
   if (t >= p.S) return false;
   if (t < p.T && p.text_mask) return p.text_mask[(long)b * p.T + t] != 0;
   return true;
 }
 
+// G query heads share one KV head; the 128-row tile holds G heads x QPOS = 128/G positions.
+template <int G, bool PREFIX>
 __global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, AttnCore p) {
@@ -84,7 +128,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   __shared__ __align__(8) uint64_t q_full;
   __shared__ __align__(8) uint64_t k_full[KV_STAGES];
   __shared__ __align__(8) uint64_t v_full[KV_STAGES];
-  __shared__ __align__(8) uint64_t kv_empty[KV_STAGES];
+  __shared__ __align__(8) uint64_t k_empty[KV_STAGES];  // freed when the S = Q K^T MMA is done
+  __shared__ __align__(8) uint64_t v_empty[KV_STAGES];  // freed when the O += P V MMA is done
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ __align__(8) uint64_t p_full;
   __shared__ __align__(8) uint64_t pv_done;
@@ -92,26 +137,49 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int n_tiles;
+  __shared__ int cta_kmin;  // PREFIX: smallest key_end of this CTA's queries (keys below it need no row mask)
   __shared__ uint16_t tiles[MAX_TILES];
 
+  constexpr int QPOS = 128 / G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p0 = blockIdx.x * QPOS, j = blockIdx.y, b = blockIdx.z;
   const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - smem_u32(smem_raw));
 
-  // ---- key tiles that hold at least one valid key (all-padded text tiles are skipped)
+  // ---- key tiles that hold at least one valid key (all-padded text tiles are skipped; with a
+  // key prefix, tiles at or beyond the largest key_end of the CTA's queries too)
   if (warp == 0) {
-    const int total = (p.S + KT - 1) / KT;
+    int kmax = p.S;
+    if constexpr (PREFIX) {
+      int hi = 0, lo = p.S;
+      for (int i = lane; i < QPOS; i += 32) {
+        const int q = p0 + i;
+        if (q < p.S) {
+          const int e = min(max(p.key_end[q], q + 1), p.S);
+          hi = max(hi, e);
+          lo = min(lo, e);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+      }
+      kmax = hi;
+      if (lane == 0) cta_kmin = lo;
+    }
+    const int total = (min(kmax, p.S) + KT - 1) / KT;
     int count = 0;
     for (int t0 = 0; t0 < total; t0 += 32) {
       const int t = t0 + lane;
       bool valid = false;
       if (t < total) {
         const int k0 = t * KT;
-        if (k0 + KT > p.T || !p.text_mask) {
-          valid = true;  // holds image keys (or no mask)
+        const int k1 = min(k0 + KT, p.S);
+        if (!p.text_mask || k1 > p.T) {
+          valid = true;  // every key valid, or the tile holds image keys (always valid)
         } else {
-          for (int k = k0; k < k0 + KT && !valid; ++k) valid = p.text_mask[(long)b * p.T + k] != 0;
+          for (int k = k0; k < k1 && !valid; ++k) valid = p.text_mask[(long)b * p.T + k] != 0;
         }
       }
       const unsigned m = __ballot_sync(0xffffffffu, valid);
@@ -125,7 +193,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
@@ -150,24 +219,38 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     if (lane == 0) {
       mbar_arrive_expect_tx(&q_full, Q_BYTES);
 #pragma unroll
-      for (int hl = 0; hl < AG; ++hl)
+      for (int hl = 0; hl < G; ++hl)
 #pragma unroll
         for (int c = 0; c < 2; ++c)
-          tma_load_3d(base + OFF_Q + c * Q_CHUNK + hl * (QPOS * 128), &tmQ, &q_full, (j * AG + hl) * AD + c * 64,
+          tma_load_3d(base + OFF_Q + c * Q_CHUNK + hl * (QPOS * 128), &tmQ, &q_full, (j * G + hl) * AD + c * 64,
                       p0, b);
-      for (int i = 0; i < n; ++i) {
+      // K tile i+1 is issued before V tile i: K stages free up as soon as their S MMA is done,
+      // V stages only after P V, so the K loads run a tile further ahead
+      auto load_k = [&](int i) -> bool {
         const int st = i % KV_STAGES;
-        const uint32_t ph = (i / KV_STAGES) & 1;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1, abort)) break;
-        const int t0 = tiles[i] * KT;
+        if (!mbar_wait(&k_empty[st], ((i / KV_STAGES) & 1) ^ 1, abort)) return false;
         uint8_t* kd = base + OFF_K + st * KV_TILE_BYTES;
-        uint8_t* vd = base + OFF_V + st * KV_TILE_BYTES;
+        const int t0 = tiles[i] * KT;
         mbar_arrive_expect_tx(&k_full[st], KV_TILE_BYTES);
         tma_load_3d(kd, &tmK, &k_full[st], j * AD, t0, b);
         tma_load_3d(kd + KV_CHUNK, &tmK, &k_full[st], j * AD + 64, t0, b);
+        return true;
+      };
+      auto load_v = [&](int i) -> bool {
+        const int st = i % KV_STAGES;
+        if (!mbar_wait(&v_empty[st], ((i / KV_STAGES) & 1) ^ 1, abort)) return false;
+        uint8_t* vd = base + OFF_V + st * KV_TILE_BYTES;
+        const int t0 = tiles[i] * KT;
         mbar_arrive_expect_tx(&v_full[st], KV_TILE_BYTES);
         tma_load_3d(vd, &tmV, &v_full[st], j * AD, t0, b);
         tma_load_3d(vd + KV_CHUNK, &tmV, &v_full[st], j * AD + 64, t0, b);
+        return true;
+      };
+      if (n > 0 && load_k(0)) {
+        for (int i = 0; i < n; ++i) {
+          if (i + 1 < n && !load_k(i + 1)) break;
+          if (!load_v(i)) break;
+        }
       }
     }
   } else if (warp == 1) {
@@ -187,7 +270,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           tc_mma_bf16_ts(tmem + O_COL, pt + kk * 8, smem_desc_sw128(sv + kk * 16 * 128, KV_CHUNK, 1024), IDESC_PV,
                          (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&pv_done);
-        tc_commit(&kv_empty[st]);
+        tc_commit(&v_empty[st]);
         return true;
       };
       if (mbar_wait(&q_full, 0, abort)) {
@@ -206,6 +289,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           }
           issued = true;
           tc_commit(&s_full[i & 1]);
+          tc_commit(&k_empty[st]);
           if (i >= 1 && !issue_pv(i - 1)) break;
         }
         if (!*abort && n > 0) issue_pv(n - 1);
@@ -218,12 +302,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       }
     }
   } else {
-    // ---- softmax warps: quarter q of the tile = query head 4j+q, rows = 32 positions
+    // ---- softmax warps: tile row r = 32 * quarter + lane holds head j*G + r / QPOS at position
+    // p0 + r % QPOS
     const int quarter = warp & 3;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    int row_kend = p.S;
+    if constexpr (PREFIX) {
+      const int r = quarter * 32 + lane;
+      const int q = p0 + r % QPOS;
+      row_kend = q < p.S ? min(max(p.key_end[q], q + 1), p.S) : p.S;
+    }
     for (int i = 0; i < n && ok; ++i) {
       const int sb = i & 1;
       if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
@@ -231,8 +322,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       const int t0 = tiles[i] * KT;
       const uint32_t sbase = tmem + lane_off + sb * KT;
       float v[KT];
-      tmem_ld32(sbase, v);
-      tmem_ld32(sbase + 32, v + 32);
+      tmem_ld64(sbase, v);
       if ((t0 < p.T && p.text_mask) || (t0 + KT > p.S)) {  // warp-uniform: only partial tiles mask
         const uint32_t vm0 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + lane));
         const uint32_t vm1 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + 32 + lane));
@@ -242,25 +332,41 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           if (!((vm1 >> e) & 1u)) v[32 + e] = -INFINITY;
         }
       }
-      float mx = v[0];
+      if constexpr (PREFIX) {
+        if (t0 + KT > cta_kmin) {  // warp-uniform; each row then cuts at its own key_end
+          const int lim = row_kend - t0;
 #pragma unroll
-      for (int e = 1; e < KT; ++e) mx = fmaxf(mx, v[e]);
+          for (int e = 0; e < KT; ++e)
+            if (e >= lim) v[e] = -INFINITY;
+        }
+      }
+      // row max: chain k takes v[k], v[k+4], ..., v[k+60] with three-input maxes
+      static_assert(KT == 64, "the max chains below cover 64 scores");
+      float m4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float a = v[k];
+#pragma unroll
+        for (int i = 1; i < 15; i += 2) a = fmax3(a, v[k + 4 * i], v[k + 4 * i + 4]);
+        m4[k] = fmaxf(a, v[k + 60]);
+      }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // exps against the running max; they only wait for the max when a row's max grows by
+      // more than 2^8 (lazy rescaling), which the warp then handles together
+      uint32_t pk[KT / 2];
+      // while a row has seen no valid key (m = -inf) its exps are taken against 0, so fully
+      // masked scores give 0 rather than NaN
+      float rs = exp_tile(v, sl2, m == -INFINITY ? 0.f : m, pk);
       const float mnew = fmaxf(m, mx * sl2);
       const bool grow = mnew > m + 8.0f;  // m = -inf on the first tile
       float alpha = 1.f;
-      if (grow) {
-        alpha = ex2(m - mnew);  // 0 on the first tile
-        m = mnew;
-      }
       const bool any_grow = __any_sync(0xffffffffu, grow);
-      uint32_t pk[KT / 2];
-      float rs = 0.f;
-#pragma unroll
-      for (int e = 0; e < KT / 2; ++e) {
-        const float a = ex2(fmaf(v[2 * e], sl2, -m));
-        const float c = ex2(fmaf(v[2 * e + 1], sl2, -m));
-        rs += a + c;
-        pk[e] = pack_bf16x2(a, c);
+      if (any_grow) {
+        if (grow) {
+          alpha = ex2(m - mnew);  // 0 on the first tile
+          m = mnew;
+        }
+        rs = exp_tile(v, sl2, m == -INFINITY ? 0.f : m, pk);
       }
       l = l * alpha + rs;
       tmem_st32(sbase, reinterpret_cast<const float*>(pk));  // P_i over the first 32 score columns
@@ -283,13 +389,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       tc_fence_before();
       mbar_arrive(&p_full);
     }
-    if (ok && n > 0 && mbar_wait(&pv_done, (n - 1) & 1, abort)) {
+    if (ok && n == 0) {
+      // a batch row without any valid key (possible only without image tokens): zeros
+      const int r = quarter * 32 + lane;
+      const int pos = p0 + r % QPOS;
+      const int h = j * G + r / QPOS;
+      if (pos < p.S) {
+        uint4* op = reinterpret_cast<uint4*>(p.out + ((long)b * p.S + pos) * p.HD + h * AD);
+#pragma unroll
+        for (int q = 0; q < AD / 8; ++q) op[q] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    } else if (ok && mbar_wait(&pv_done, (n - 1) & 1, abort)) {
       tc_fence_after();
-      const int pos = p0 + lane;
-      const int h = j * AG + quarter;
+      const int r = quarter * 32 + lane;
+      const int pos = p0 + r % QPOS;
+      const int h = j * G + r / QPOS;
       const bool row_ok = pos < p.S;
       const long grow_idx = (long)b * p.S + pos;
-      const float inv_l = 1.f / l;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no readable key: zeros
 #pragma unroll 1
       for (int c = 0; c < AD / 32; ++c) {
         float o[32];
@@ -365,14 +482,21 @@ __global__ void __launch_bounds__(256) qk_prep_kernel(const __nv_bfloat16* __res
 
 KREA2_DEFINE_ERROR_READER(take_device_error_attention)
 
-bool attention_tc_supported(int D, int H, int Hkv) { return D == AD && Hkv > 0 && H == AG * Hkv; }
+bool attention_tc_supported(int D, int H, int Hkv) {
+  if (D != AD || Hkv <= 0 || H % Hkv) return false;
+  const int g = H / Hkv;
+  return g == 1 || g == 2 || g == 4;
+}
 
-int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
+namespace {
+template <int G, bool PREFIX>
+int launch_attention_g(const AttnTcArgs& a, cudaStream_t stream) {
+  constexpr int QPOS = 128 / G;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(attn_gqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
+    if (cudaFuncSetAttribute(attn_gqa_tc_kernel<G, PREFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(attn_gqa_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+        cudaFuncSetAttribute(attn_gqa_tc_kernel<G, PREFIX>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(attention) failed");
     attr_done = true;
@@ -391,12 +515,30 @@ int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
   p.g_stride = a.g_stride;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)AD);
+  p.key_end = a.key_end;
   dim3 grid((S + QPOS - 1) / QPOS, a.Hkv, a.B);
-  attn_gqa_tc_kernel<<<grid, ATT_THREADS, ATT_SMEM, stream>>>(tq, tk, tv, p);
+  attn_gqa_tc_kernel<G, PREFIX><<<grid, ATT_THREADS, ATT_SMEM, stream>>>(tq, tk, tv, p);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
   return KREA2_OK;
+}
+}  // namespace
+
+int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
+  if (!attention_tc_supported(AD, a.H, a.Hkv)) return set_error(KREA2_ERR_UNSUPPORTED, "attention group size");
+  if (a.key_end) {
+    switch (a.H / a.Hkv) {
+      case 1: return launch_attention_g<1, true>(a, stream);
+      case 2: return launch_attention_g<2, true>(a, stream);
+      default: return launch_attention_g<4, true>(a, stream);
+    }
+  }
+  switch (a.H / a.Hkv) {
+    case 1: return launch_attention_g<1, false>(a, stream);
+    case 2: return launch_attention_g<2, false>(a, stream);
+    default: return launch_attention_g<4, false>(a, stream);
+  }
 }
 
 int launch_qk_prep(const void* qkvg, long long stride, int B, int S, int H, int Hkv, float eps, const float* qw,

@@ -191,6 +191,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
+          if (p.bias) {
+            const float4* bp = reinterpret_cast<const float4*>(p.bias + (size_t)nt * BN + c * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 bv = __ldg(bp + q);
+              v[q * 4 + 0] += bv.x;
+              v[q * 4 + 1] += bv.y;
+              v[q * 4 + 2] += bv.z;
+              v[q * 4 + 3] += bv.w;
+            }
+          }
           if (row_ok) {
             uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
@@ -246,43 +257,51 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           const bool is_k = !is_q && c0 < p.HD + p.KVD;
           const uint32_t ub = tbase + u * 128;
           float r = 1.f;
-          const float* w = is_q ? p.qw : p.kw;
-          if (is_q || is_k) {
-            float ss = 0.f;
+          if (is_q || is_k) {  // pass 1: sum of squares over the head's 128 columns
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              float v[32];
-              tmem_ld32(ub + c * 32, v);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              float v[64];
+              tmem_ld64(ub + h2 * 64, v);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ss += v[e] * v[e];
+              for (int e = 0; e < 64; ++e) s4[e & 3] += v[e] * v[e];
             }
-            r = rsqrtf(ss * (1.f / 128.f) + p.eps);
+            r = rsqrtf(((s4[0] + s4[1]) + (s4[2] + s4[3])) * (1.f / 128.f) + p.eps);
           }
+          const float4* w4 = reinterpret_cast<const float4*>(is_q ? p.qw : p.kw);
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float v[32];
-            tmem_ld32(ub + c * 32, v);
+          for (int h2 = 0; h2 < 2; ++h2) {  // pass 2: normalise, rotate, store 64 columns at a time
+            float v[64];
+            tmem_ld64(ub + h2 * 64, v);
             if (is_q || is_k) {
+              const float4* c4 = reinterpret_cast<const float4*>(cs + h2 * 32);
+              const float4* s4p = reinterpret_cast<const float4*>(sn + h2 * 32);
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                const int d = c * 32 + e;
-                const float x0 = v[e] * r * (1.f + __ldg(w + d));
-                const float x1 = v[e + 1] * r * (1.f + __ldg(w + d + 1));
-                const float co = __ldg(cs + d / 2), si = __ldg(sn + d / 2);
-                v[e] = x0 * co - x1 * si;
-                v[e + 1] = x1 * co + x0 * si;
+              for (int q = 0; q < 8; ++q) {  // 8 dims (4 rotated pairs) per step
+                const float4 wa = __ldg(w4 + h2 * 16 + 2 * q), wb = __ldg(w4 + h2 * 16 + 2 * q + 1);
+                const float4 co = __ldg(c4 + q), si = __ldg(s4p + q);
+                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                const float cv[4] = {co.x, co.y, co.z, co.w}, sv[4] = {si.x, si.y, si.z, si.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int d = q * 8 + 2 * e;
+                  const float x0 = v[d] * r * (1.f + wv[2 * e]);
+                  const float x1 = v[d + 1] * r * (1.f + wv[2 * e + 1]);
+                  v[d] = x0 * cv[e] - x1 * sv[e];
+                  v[d + 1] = x1 * cv[e] + x0 * sv[e];
+                }
               }
             }
             if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + u * 128 + c * 32);
+              uint4* dst = reinterpret_cast<uint4*>(out + u * 128 + h2 * 64);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint4 w4;
-                w4.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-                w4.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-                w4.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-                w4.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-                dst[q] = w4;
+              for (int q = 0; q < 8; ++q) {
+                uint4 w4o;
+                w4o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
+                w4o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
+                w4o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
+                w4o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
+                dst[q] = w4o;
               }
             }
           }

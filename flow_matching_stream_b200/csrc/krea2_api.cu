@@ -1,5 +1,6 @@
 // C ABI entry points (include/krea2.h): argument checks, workspace carving and the launch
 // sequence of the block and the backbone. Every step runs in this library's kernels.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -67,6 +68,7 @@ int check_dims(const Krea2Dims* d, int dtype) {
 int check_model_dims(const Krea2Dims* d) {
   if (d->n_layers < 0) return set_error(KREA2_ERR_ARG, "n_layers < 0");
   if (d->in_ch <= 0) return set_error(KREA2_ERR_ARG, "in_ch must be positive");
+  if (d->in_ch > 64) return set_error(KREA2_ERR_UNSUPPORTED, "in_ch must be <= 64");
   if (d->t_dim <= 0 || d->t_dim % 8 || d->t_dim > d->C)
     return set_error(KREA2_ERR_UNSUPPORTED, "t_dim must be a positive multiple of 8 and <= C");
   return KREA2_OK;
@@ -84,7 +86,7 @@ constexpr size_t ALIGN = 256;
 inline size_t up(size_t x) { return (x + ALIGN - 1) & ~(ALIGN - 1); }
 
 struct Ws {
-  size_t mod, xn, qkvg, attn, u, h, cs, sn, temb, e, tscr, ybuf, total;
+  size_t mod, xn, qkvg, attn, u, h, cs, sn, temb, e, tscr, total;
 };
 
 Ws ws_layout(const Krea2Dims* d, int B, int T, int N, int dtype) {
@@ -109,14 +111,13 @@ Ws ws_layout(const Krea2Dims* d, int B, int T, int N, int dtype) {
   w.temb = take((size_t)B * 6 * C * 4);
   w.e = take((size_t)B * C * 4);
   w.tscr = take((size_t)B * C * 4);
-  w.ybuf = take((size_t)B * N * C * 4);
   w.total = off;
   return w;
 }
 
 // Standalone attention on raw projection columns ([ARCH] §四.3): the tensor-core path first
 // writes normalised, rotated q|k into the workspace, then runs the flash-attention core.
-int attention_raw(const AttnParams& p, int dtype, void* ws, cudaStream_t s) {
+int attention_raw(const AttnParams& p, int dtype, void* ws, cudaStream_t s, const int* key_end = nullptr) {
   if (dtype == KREA2_BF16 && attention_tc_supported(p.D, p.H, p.Hkv)) {
     const long long QC = 2LL * p.H * p.D + 2LL * p.Hkv * p.D;
     int rc = launch_qk_prep(p.qkvg, QC, p.B, p.S, p.H, p.Hkv, p.eps, p.q_norm_w, p.k_norm_w, p.cos, p.sin, ws, s);
@@ -130,9 +131,10 @@ int attention_raw(const AttnParams& p, int dtype, void* ws, cudaStream_t s) {
     a.k = prep + (long long)p.H * p.D; a.k_stride = QK;
     a.v = raw + (long long)(p.H + p.Hkv) * p.D; a.v_stride = QC;
     a.g = raw + (long long)(p.H + 2 * p.Hkv) * p.D; a.g_stride = QC;
-    a.text_mask = p.text_mask; a.out = p.out;
+    a.text_mask = p.text_mask; a.out = p.out; a.key_end = key_end;
     return attention_tc_core(a, s);
   }
+  if (key_end) return set_error(KREA2_ERR_UNSUPPORTED, "block-causal attention needs bf16, D=128, H/Hkv in {1,2,4}");
   return attention_simt(p, dtype == KREA2_BF16, s);
 }
 
@@ -193,7 +195,10 @@ int block_impl(const Krea2Dims* d, int B, int T, int N, int dtype, float* h, con
   void* u = ws + L.u;
   int rc;
   mark(0);
-  if ((rc = launch_modulation(temb, w->scale_shift_table, B, C, mod, s))) return rc;
+  // no table: a block without time modulation (text fusion): scale 0, shift 0, gate 1
+  if ((rc = w->scale_shift_table ? launch_modulation(temb, w->scale_shift_table, B, C, mod, s)
+                                 : launch_unit_modulation(B, C, mod, s)))
+    return rc;
   mark(1);
   if ((rc = launch_mod_rmsnorm(h, w->norm1_w, mod, nullptr, 0, B, S, C, d->eps, xn, bf, s))) return rc;
   if (bf && attention_tc_supported(d->D, d->H, d->Hkv)) {
@@ -295,6 +300,49 @@ int krea2_gqa_attention(const Krea2Dims* dims, int B, int T, int N, int dtype, c
   return attention_raw(ap, dtype, workspace, as_stream(stream));
 }
 
+int krea2_block_causal_key_end(const int32_t* image_ids, int S, int32_t* key_end) {
+  if (!image_ids || !key_end || S <= 0) return set_error(KREA2_ERR_ARG, "NULL pointer or S <= 0");
+  int end = 0;
+  for (int q = S - 1; q >= 0; --q) {  // image ids run contiguously; walk back to know each block's end
+    const int id = image_ids[q];
+    if (id < 0) {
+      key_end[q] = q + 1;
+      continue;
+    }
+    if (q == S - 1 || image_ids[q + 1] != id) end = q + 1;
+    key_end[q] = end;
+  }
+  for (int q = 0; q < S; ++q)  // a block id appearing in two separated runs is not a block
+    if (image_ids[q] >= 0 && (q == 0 || image_ids[q - 1] != image_ids[q]))
+      for (int k = key_end[q]; k < S; ++k)
+        if (image_ids[k] == image_ids[q]) return set_error(KREA2_ERR_ARG, "image block %d is not contiguous", image_ids[q]);
+  return KREA2_OK;
+}
+
+int krea2_gqa_attention_block_causal(const Krea2Dims* dims, int B, int T, int N, int dtype, const void* qkvg,
+                                     const float* q_norm_w, const float* k_norm_w, const float* cos,
+                                     const float* sin, const uint8_t* text_mask, const int32_t* key_end, void* out,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc) return rc;
+  // every query reads at least its own position, so (unlike the plain entry) no image token is
+  // needed; a query whose readable keys are all padded outputs zeros
+  if (B <= 0 || T < 0 || N < 0 || T + N <= 0) return set_error(KREA2_ERR_ARG, "need B >= 1 and T + N >= 1");
+  if (!qkvg || !q_norm_w || !k_norm_w || !cos || !sin || !out || !key_end)
+    return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (dtype != KREA2_BF16 || !attention_tc_supported(dims->D, dims->H, dims->Hkv))
+    return set_error(KREA2_ERR_UNSUPPORTED, "block-causal attention needs bf16, D=128, H/Hkv in {1,2,4}");
+  const size_t need = attention_ws_bytes(dims, B, T, N, dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (ws_bytes < need) return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  AttnParams ap{};
+  ap.B = B; ap.T = T; ap.N = N; ap.S = T + N; ap.H = dims->H; ap.Hkv = dims->Hkv; ap.D = dims->D;
+  ap.eps = dims->eps; ap.qkvg = qkvg; ap.q_norm_w = q_norm_w; ap.k_norm_w = k_norm_w; ap.cos = cos; ap.sin = sin;
+  ap.text_mask = T > 0 ? text_mask : nullptr; ap.out = out;
+  return attention_raw(ap, dtype, workspace, as_stream(stream), key_end);
+}
+
 int krea2_modulated_rmsnorm(const Krea2Dims* dims, int B, int S, int dtype, const float* h, const float* norm_w,
                             const float* temb, const float* table, int chunk, void* out, void* stream) {
   int rc = check_dims(dims, dtype);
@@ -333,12 +381,12 @@ int krea2_time_embed(const Krea2Dims* dims, int B, int dtype, const float* times
 }
 
 int krea2_final_layer(const Krea2Dims* dims, int B, int T, int N, int dtype, const float* h, const float* e,
-                      const Krea2ModelWeights* w, void* velocity, float* scratch, void* stream) {
+                      const Krea2ModelWeights* w, void* velocity, void* stream) {
   int rc = check_dims(dims, dtype);
   if (rc || (rc = check_model_dims(dims)) || (rc = check_shape(B, T, N))) return rc;
-  if (!h || !e || !w || !w->final_norm_w || !w->final_table || !w->final_w || !w->final_b || !velocity || !scratch)
+  if (!h || !e || !w || !w->final_norm_w || !w->final_table || !w->final_w || !w->final_b || !velocity)
     return set_error(KREA2_ERR_ARG, "NULL pointer");
-  return launch_final_layer(dims, B, T, N, dtype == KREA2_BF16, h, e, w, scratch, velocity, as_stream(stream));
+  return launch_final_layer(dims, B, T, N, dtype == KREA2_BF16, h, e, w, velocity, as_stream(stream));
 }
 
 int krea2_block_forward(const Krea2Dims* dims, int B, int T, int N, int dtype, float* h, const float* temb,
@@ -376,6 +424,223 @@ int krea2_block_forward_traced(const Krea2Dims* dims, int B, int T, int N, int d
 
 unsigned long long krea2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+namespace {
+Krea2Dims text_block_dims(const Krea2TextDims* td) {
+  Krea2Dims d{};
+  d.C = td->Dt; d.H = td->H; d.Hkv = td->Hkv; d.D = td->D; d.F = td->F;
+  d.axes[0] = td->D / 4; d.axes[1] = 3 * td->D / 8; d.axes[2] = td->D - d.axes[0] - d.axes[1];
+  d.theta = 1000.f; d.eps = td->eps; d.n_layers = 0; d.in_ch = 1; d.t_dim = 8;
+  return d;
+}
+
+int check_text_dims(const Krea2TextDims* td, int dtype, int B, int T) {
+  if (!td) return set_error(KREA2_ERR_ARG, "text dims is NULL");
+  if (td->L <= 0 || td->n_layerwise < 0 || td->n_refiner < 0 || td->C <= 0 || td->C % 128)
+    return set_error(KREA2_ERR_ARG, "bad text-fusion dims");
+  if (B <= 0 || T <= 0) return set_error(KREA2_ERR_ARG, "need B >= 1 and T >= 1");
+  const Krea2Dims d = text_block_dims(td);
+  return check_dims(&d, dtype);
+}
+
+struct TextWs {
+  size_t hl, hr, cs, sn, proj, block, total;
+};
+TextWs text_layout(const Krea2TextDims* td, int B, int T, int dtype) {
+  const Krea2Dims d = text_block_dims(td);
+  const size_t es = dtype == KREA2_BF16 ? 2 : 4;
+  TextWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += up(bytes);
+    return o;
+  };
+  const size_t rows_l = (size_t)B * T * td->L;
+  w.hl = take(rows_l * td->Dt * 4);
+  w.hr = take((size_t)B * T * td->Dt * 4);
+  const size_t smax = (size_t)(T > td->L ? T : td->L);
+  w.cs = take(smax * (td->D / 2) * 4);
+  w.sn = take(smax * (td->D / 2) * 4);
+  w.proj = take((size_t)B * T * td->Dt * es);
+  const size_t b1 = ws_layout(&d, B * T, 0, td->L, dtype).total, b2 = ws_layout(&d, B, T, 0, dtype).total;
+  w.block = take(b1 > b2 ? b1 : b2);
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+size_t krea2_text_fusion_workspace_size(const Krea2TextDims* td, int B, int T, int dtype) {
+  if (check_text_dims(td, dtype, B, T)) return 0;
+  return text_layout(td, B, T, dtype).total;
+}
+
+int krea2_text_fusion(const Krea2TextDims* td, int B, int T, int dtype, const void* ehs, const uint8_t* text_mask,
+                      const Krea2TextWeights* w, void* text_out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_text_dims(td, dtype, B, T);
+  if (rc) return rc;
+  if (!ehs || !w || !text_out || !w->layer_w || !w->txt_in_w || !w->txt_in_b ||
+      (td->n_layerwise && !w->layerwise) || (td->n_refiner && !w->refiner))
+    return set_error(KREA2_ERR_ARG, "NULL pointer");
+  for (int i = 0; i < td->n_layerwise + td->n_refiner; ++i) {
+    const Krea2BlockWeights* b = i < td->n_layerwise ? &w->layerwise[i] : &w->refiner[i - td->n_layerwise];
+    if (!b->w_qkvg || !b->w_out || !b->w_gu || !b->w_down || !b->norm1_w || !b->norm2_w || !b->q_norm_w ||
+        !b->k_norm_w)
+      return set_error(KREA2_ERR_ARG, "text-fusion block %d: NULL pointer", i);
+    if (b->scale_shift_table) return set_error(KREA2_ERR_ARG, "text-fusion blocks take no modulation table");
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const TextWs L = text_layout(td, B, T, dtype);
+  if (ws_bytes < L.total) return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  const Krea2Dims d = text_block_dims(td);
+  const bool bf = dtype == KREA2_BF16;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  float* hl = reinterpret_cast<float*>(ws + L.hl);
+  float* hr = reinterpret_cast<float*>(ws + L.hr);
+  float* cs = reinterpret_cast<float*>(ws + L.cs);
+  float* sn = reinterpret_cast<float*>(ws + L.sn);
+  const int smax = T > td->L ? T : td->L;
+  // no RoPE anywhere in text fusion: the zero-position (identity) rotation
+  if ((rc = launch_identity_rope((long)smax * (td->D / 2), cs, sn, s))) return rc;
+  // 1. layerwise: B*T sequences of L layer tokens, no mask
+  const long rows_l = (long)B * T * td->L;
+  if ((rc = launch_to_f32(ehs, bf, rows_l * td->Dt, hl, s))) return rc;
+  const Ws bl = ws_layout(&d, B * T, 0, td->L, dtype);
+  for (int i = 0; i < td->n_layerwise; ++i)
+    if ((rc = block_impl(&d, B * T, 0, td->L, dtype, hl, nullptr, &w->layerwise[i], cs, sn, nullptr, ws + L.block,
+                         bl, s)))
+      return rc;
+  // 2. Linear(L, 1) over the layer axis
+  if ((rc = launch_layer_projection(hl, w->layer_w, (long)B * T, td->L, td->Dt, hr, false, s))) return rc;
+  // 3. refiner over the token sequence with the text mask (T "text" keys, no image keys)
+  const Ws br = ws_layout(&d, B, T, 0, dtype);
+  for (int i = 0; i < td->n_refiner; ++i)
+    if ((rc = block_impl(&d, B, T, 0, dtype, hr, nullptr, &w->refiner[i], cs, sn, text_mask, ws + L.block, br, s)))
+      return rc;
+  // 4. txt_in: Linear(Dt, C) + bias
+  void* proj = ws + L.proj;
+  if ((rc = launch_to_dtype(hr, (long)B * T * td->Dt, proj, bf, s))) return rc;
+  if (bf) {
+    GemmParams gp{};
+    gp.M = B * T; gp.N = td->C; gp.K = td->Dt; gp.out = text_out; gp.bias = w->txt_in_b;
+    return gemm_bf16(EPI_STORE, gp, proj, w->txt_in_w, s);
+  }
+  SimtGemmParams sp{};
+  sp.M = B * T; sp.N = td->C; sp.K = td->Dt; sp.out = text_out; sp.bias = w->txt_in_b;
+  return gemm_simt(SEPI_BIAS_F32, sp, proj, false, w->txt_in_w, false, s);
+}
+
+double krea2_shift_mu(int image_seq_len) {
+  const double base_len = 256.0, max_len = 6400.0, base_shift = 0.5, max_shift = 1.15;
+  return base_shift + (max_shift - base_shift) / (max_len - base_len) * ((double)image_seq_len - base_len);
+}
+
+int krea2_sigma_schedule(int n_steps, double mu, float* sigmas_out) {
+  if (n_steps < 1 || !sigmas_out) return set_error(KREA2_ERR_ARG, "need n_steps >= 1 and an output array");
+  const double em = exp(mu);
+  for (int i = 0; i < n_steps; ++i) {
+    // linspace(1, 1/n, n)
+    const double s = n_steps == 1 ? 1.0 : 1.0 + (1.0 / n_steps - 1.0) * (double)i / (double)(n_steps - 1);
+    sigmas_out[i] = (float)(em / (em + (1.0 / s - 1.0)));
+  }
+  sigmas_out[n_steps] = 0.f;
+  return KREA2_OK;
+}
+
+int krea2_euler_cfg_step(int dtype, long long n, float* x, const void* v_cond, const void* v_uncond, float guidance,
+                         float sigma, float sigma_next, void* x_model, int copies, float* timestep_out,
+                         void* stream) {
+  if (dtype != KREA2_BF16 && dtype != KREA2_F32) return set_error(KREA2_ERR_ARG, "unknown dtype %d", dtype);
+  if (n < 0 || !x || !v_cond) return set_error(KREA2_ERR_ARG, "NULL pointer or negative size");
+  if ((x_model || timestep_out) && (copies < 1 || copies > 32)) return set_error(KREA2_ERR_ARG, "copies must be 1..32");
+  return launch_euler_cfg(dtype == KREA2_BF16, n, x, v_cond, guidance > 0.f ? v_uncond : nullptr, guidance, sigma,
+                          sigma_next, x_model, copies, timestep_out, as_stream(stream));
+}
+
+namespace {
+struct SampleWs {
+  size_t backbone, backbone_bytes, xin, text, mask, t, vel, total;
+};
+SampleWs sample_layout(const Krea2Dims* d, int T, int N, int dtype, int cfg) {
+  const int B = cfg ? 2 : 1;
+  const size_t es = dtype == KREA2_BF16 ? 2 : 4;
+  SampleWs w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += up(bytes);
+    return o;
+  };
+  w.backbone_bytes = ws_layout(d, B, T, N, dtype).total;
+  w.backbone = take(w.backbone_bytes);
+  w.xin = take((size_t)B * N * d->in_ch * es);
+  w.text = take((size_t)B * T * d->C * es + 16);
+  w.mask = take((size_t)B * T + 16);
+  w.t = take((size_t)B * 4);
+  w.vel = take((size_t)B * N * d->in_ch * es);
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+size_t krea2_sample_workspace_size(const Krea2Dims* dims, int T, int N, int dtype, int cfg) {
+  if (check_dims(dims, dtype) || check_model_dims(dims) || check_shape(1, T, N)) return 0;
+  return sample_layout(dims, T, N, dtype, cfg).total;
+}
+
+int krea2_sample(const Krea2Dims* dims, int T, int N, int dtype, float* latents, const void* text_cond,
+                 const void* text_uncond, const uint8_t* mask_cond, const uint8_t* mask_uncond,
+                 const float* position_ids, const float* sigmas, int n_steps, float guidance,
+                 const Krea2ModelWeights* w, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc || (rc = check_model_dims(dims)) || (rc = check_shape(1, T, N)) ||
+      (rc = check_model_weights(w, dims->n_layers)))
+    return rc;
+  const bool cfg = guidance > 0.f;
+  if (!latents || (T > 0 && !text_cond) || (cfg && T > 0 && !text_uncond) || !position_ids || !sigmas || n_steps < 1)
+    return set_error(KREA2_ERR_ARG, "NULL pointer or n_steps < 1");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  const SampleWs L = sample_layout(dims, T, N, dtype, cfg);
+  if (ws_bytes < L.total) return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L.total);
+  const int B = cfg ? 2 : 1;
+  const bool bf = dtype == KREA2_BF16;
+  const size_t es = bf ? 2 : 4;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  void* xin = ws + L.xin;
+  void* text = ws + L.text;
+  uint8_t* mask = ws + L.mask;
+  float* tt = reinterpret_cast<float*>(ws + L.t);
+  void* vel = ws + L.vel;
+  const size_t text_bytes = (size_t)T * dims->C * es;
+  // batch rows [cond, uncond]: text, masks (NULL = all valid)
+  if (T > 0) {
+    cudaError_t e = cudaMemcpyAsync(text, text_cond, text_bytes, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess && cfg)
+      e = cudaMemcpyAsync(reinterpret_cast<uint8_t*>(text) + text_bytes, text_uncond, text_bytes,
+                          cudaMemcpyDeviceToDevice, s);
+    for (int r = 0; r < B && e == cudaSuccess; ++r) {
+      const uint8_t* m = r == 0 ? mask_cond : mask_uncond;
+      e = m ? cudaMemcpyAsync(mask + (size_t)r * T, m, T, cudaMemcpyDeviceToDevice, s)
+            : cudaMemsetAsync(mask + (size_t)r * T, 1, T, s);
+    }
+    if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "staging the text batch failed: %s", cudaGetErrorString(e));
+  }
+  const long long n = (long long)N * dims->in_ch;
+  // first model input: x at sigmas[0]
+  if ((rc = launch_euler_cfg(bf, n, latents, nullptr, nullptr, 0.f, sigmas[0], sigmas[0], xin, B, tt, s))) return rc;
+  for (int i = 0; i < n_steps; ++i) {
+    if ((rc = krea2_backbone_forward(dims, B, T, N, dtype, xin, text, position_ids, T > 0 ? mask : nullptr, tt, w, vel,
+                                     ws + L.backbone, L.backbone_bytes, stream)))
+      return rc;
+    const void* vu = cfg ? reinterpret_cast<uint8_t*>(vel) + (size_t)n * es : nullptr;
+    if ((rc = launch_euler_cfg(bf, n, latents, vel, vu, guidance, sigmas[i], sigmas[i + 1], xin, B, tt, s))) return rc;
+  }
+  return KREA2_OK;
+}
+
 int krea2_backbone_forward(const Krea2Dims* dims, int B, int T, int N, int dtype, const void* hidden_states,
                            const void* text_states, const float* position_ids, const uint8_t* text_mask,
                            const float* timestep, const Krea2ModelWeights* w, void* velocity, void* workspace,
@@ -411,7 +676,7 @@ int krea2_backbone_forward(const Krea2Dims* dims, int B, int T, int N, int dtype
   const uint8_t* mask = T > 0 ? text_mask : nullptr;
   for (int l = 0; l < dims->n_layers; ++l)
     if ((rc = block_impl(dims, B, T, N, dtype, h, temb, &w->blocks[l], cs, sn, mask, ws, L, s))) return rc;
-  return launch_final_layer(dims, B, T, N, bf, h, e, w, reinterpret_cast<float*>(ws + L.ybuf), velocity, s);
+  return launch_final_layer(dims, B, T, N, bf, h, e, w, velocity, s);
 }
 
 }  // extern "C"

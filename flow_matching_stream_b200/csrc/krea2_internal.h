@@ -22,6 +22,7 @@ int take_device_error_attention();
 struct GemmParams {
   int M, N, K;              // N = rows of W
   void* out;                // STORE/SWIGLU: bf16 (M, N) / (M, N/2); RESID: fp32 (M, N)
+  const float* bias;        // STORE: optional per-column bias (N)
   const float* gate;        // RESID: gate[(row / rows_per_batch) * gate_stride + col]
   int rows_per_batch;       // RESID: batch of a row; QKV: sequence length S (position = row % S)
   long long gate_stride;
@@ -67,7 +68,15 @@ int launch_mod_rmsnorm(const float* h, const float* w, const float* temb, const 
 int launch_time_embed(const Krea2Dims* d, int B, bool w_bf16, const float* t, const Krea2ModelWeights* w,
                       float* temb, float* e, float* scratch, cudaStream_t stream);
 int launch_final_layer(const Krea2Dims* d, int B, int T, int N, bool bf16, const float* h, const float* e,
-                       const Krea2ModelWeights* w, float* ybuf, void* velocity, cudaStream_t stream);
+                       const Krea2ModelWeights* w, void* velocity, cudaStream_t stream);
+int launch_euler_cfg(bool bf16, long long n, float* x, const void* vc, const void* vu, float g, float sigma,
+                     float sigma_next, void* xm, int copies, float* t_out, cudaStream_t stream);
+int launch_unit_modulation(int B, int C, float* mod, cudaStream_t stream);
+int launch_identity_rope(long n, float* cs, float* sn, cudaStream_t stream);
+int launch_layer_projection(const float* x, const float* w, long rows, int L, int C, void* out, bool out_bf16,
+                            cudaStream_t stream);
+int launch_to_f32(const void* in, bool in_bf16, long n, float* out, cudaStream_t stream);
+int launch_to_dtype(const float* in, long n, void* out, bool out_bf16, cudaStream_t stream);
 int launch_copy_text_rows(const void* text, bool bf16, int B, int T, int S, int C, float* h, cudaStream_t stream);
 
 // Attention (attention_*.cu).
@@ -93,6 +102,7 @@ struct AttnTcArgs {
   const void* g; long long g_stride;
   const uint8_t* text_mask;
   void* out;                           // (B*S, H*128) bf16
+  const int* key_end;                  // optional (S): query q reads keys [0, key_end[q]) (block-causal)
 };
 bool attention_tc_supported(int D, int H, int Hkv);
 int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream);

@@ -51,6 +51,54 @@ __global__ void modulation_kernel(const float* __restrict__ temb, const float* _
     mod[i] = temb[i] + table[i % (6L * C)];
 }
 
+// Unit modulation (scale 0, shift 0, gate 1 for both halves): blocks without time modulation.
+__global__ void unit_modulation_kernel(int B, int C, float* __restrict__ mod) {
+  const long n = (long)B * 6 * C;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const int chunk = (int)((i / C) % 6);
+    mod[i] = (chunk == 2 || chunk == 5) ? 1.f : 0.f;
+  }
+}
+
+// RoPE tables of the zero position: cos 1, sin 0 (the identity rotation).
+__global__ void identity_rope_kernel(long n, float* __restrict__ cs, float* __restrict__ sn) {
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    cs[i] = 1.f;
+    sn[i] = 0.f;
+  }
+}
+
+// out[n, c] = sum_l w[l] * x[n*L + l, c]   (Linear(L, 1, bias=False) over the layer axis)
+template <bool OUT_BF16>
+__global__ void layer_projection_kernel(const float* __restrict__ x, const float* __restrict__ w, long rows, int L,
+                                        int C, void* __restrict__ out) {
+  const long total = rows * C;
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const long r = i / C;
+    const int c = (int)(i % C);
+    float acc = 0.f;
+    for (int l = 0; l < L; ++l) acc += w[l] * x[(r * L + l) * C + c];
+    if (OUT_BF16) reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(acc);
+    else reinterpret_cast<float*>(out)[i] = acc;
+  }
+}
+
+// fp32 copy of an activation tensor in `dtype`
+template <bool IN_BF16>
+__global__ void to_f32_kernel(const void* __restrict__ in, long n, float* __restrict__ out) {
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+    out[i] = IN_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(in)[i])
+                     : reinterpret_cast<const float*>(in)[i];
+}
+
+template <bool OUT_BF16>
+__global__ void from_f32_kernel(const float* __restrict__ in, long n, void* __restrict__ out) {
+  for (long i = (long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    if (OUT_BF16) reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(in[i]);
+    else reinterpret_cast<float*>(out)[i] = in[i];
+  }
+}
+
 // ----------------------------------------------------------------------------- modulated RMSNorm
 // One CTA per row; C % 4 == 0; 256 threads, float4 loads of the fp32 residual.
 template <bool OUT_BF16>
@@ -180,29 +228,86 @@ __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __rest
   }
 }
 
-// ----------------------------------------------------------------------------- final layer prologue
-// y[b*N + n] = (1 + table[0] + e[b]) * rms(h[b*S + T + n]) * (1 + w) + (table[1] + e[b])
-__global__ void __launch_bounds__(256) final_norm_kernel(const float* __restrict__ h, const float* __restrict__ e,
-                                                         const float* __restrict__ w,
-                                                         const float* __restrict__ table, int T, int N, int S, int C,
-                                                         float eps, float* __restrict__ y) {
-  const long r = blockIdx.x;  // 0 .. B*N-1
-  const int b = (int)(r / N), n = (int)(r % N);
-  const float* x = h + ((long)b * S + T + n) * C;
-  float ss = 0.f;
-  for (int c = threadIdx.x; c < C; c += 256) ss += x[c] * x[c];
-  __shared__ float red[8];
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+// ----------------------------------------------------------------------------- final layer
+// velocity[b*N + n] = ((1 + table[0] + e[b]) * rms(h[b*S + T + n]) * (1 + w) + table[1] + e[b]) . Wfᵀ + bias
+// One CTA per FL_ROWS image rows: the row statistics first, then K-chunks of the modulated rows
+// and of Wf staged in shared memory; each thread accumulates FL_ROWS*OUT/256 outputs.
+constexpr int FL_ROWS = 16, FL_KC = 128, FL_MAX_OUT = 64;
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) final_layer_kernel(const float* __restrict__ h, const float* __restrict__ e,
+                                                          const float* __restrict__ w, const float* __restrict__ table,
+                                                          const void* __restrict__ Wf, const float* __restrict__ bias,
+                                                          int B, int T, int N, int C, int OUT, float eps,
+                                                          void* __restrict__ velocity) {
+  __shared__ float xs[FL_ROWS][FL_KC + 1];
+  __shared__ float ws[FL_MAX_OUT][FL_KC + 1];
+  __shared__ float rr[FL_ROWS];
+  const int S = T + N;
+  const long r0 = (long)blockIdx.x * FL_ROWS;
+  const long rows = (long)B * N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // row statistics: 8 warps x 2 rows
+  for (int i = warp; i < FL_ROWS; i += 8) {
+    const long r = r0 + i;
+    float ss = 0.f;
+    if (r < rows) {
+      const float* x = h + ((r / N) * S + T + (r % N)) * (long)C;
+      for (int c = lane; c < C; c += 32) ss += x[c] * x[c];
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) rr[i] = rsqrtf(ss / (float)C + eps);
+  }
+  // each thread: row tr, outputs to .. to + OPT-1
+  constexpr int THREADS_PER_ROW = 256 / FL_ROWS;  // 16
+  const int tr = threadIdx.x / THREADS_PER_ROW;
+  const int opt = (OUT + THREADS_PER_ROW - 1) / THREADS_PER_ROW;  // <= 4
+  const int to = (threadIdx.x % THREADS_PER_ROW) * opt;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
   __syncthreads();
-  float tot = 0.f;
-  for (int i = 0; i < 8; ++i) tot += red[i];
-  const float rr = rsqrtf(tot / (float)C + eps);
-  const float* eb = e + (long)b * C;
-  for (int c = threadIdx.x; c < C; c += 256) {
-    const float sc = table[c] + eb[c];
-    const float sh = table[C + c] + eb[c];
-    y[r * C + c] = (1.f + sc) * (x[c] * rr * (1.f + w[c])) + sh;
+  for (int k0 = 0; k0 < C; k0 += FL_KC) {
+    for (int i = threadIdx.x; i < FL_ROWS * FL_KC; i += 256) {
+      const int rl = i / FL_KC, k = i % FL_KC;
+      const long r = r0 + rl;
+      const int c = k0 + k;
+      float y = 0.f;
+      if (r < rows && c < C) {
+        const long b = r / N;
+        const float x = h[(b * S + T + (r % N)) * (long)C + c];
+        const float sc = table[c] + e[b * C + c], sh = table[C + c] + e[b * C + c];
+        y = (1.f + sc) * (x * rr[rl] * (1.f + w[c])) + sh;
+      }
+      xs[rl][k] = y;
+    }
+    for (int i = threadIdx.x; i < OUT * FL_KC; i += 256) {
+      const int o = i / FL_KC, k = i % FL_KC;
+      const int c = k0 + k;
+      float v = 0.f;
+      if (c < C) {
+        v = BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(Wf)[(long)o * C + c])
+                 : reinterpret_cast<const float*>(Wf)[(long)o * C + c];
+      }
+      ws[o][k] = v;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int k = 0; k < FL_KC; ++k) {
+      const float a = xs[tr][k];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < opt && to + q < OUT) acc[q] += a * ws[to + q][k];
+    }
+    __syncthreads();
+  }
+  const long r = r0 + tr;
+  if (r < rows) {
+    for (int q = 0; q < opt; ++q) {
+      const int o = to + q;
+      if (o >= OUT) break;
+      const float v = acc[q] + bias[o];
+      if (BF16) reinterpret_cast<__nv_bfloat16*>(velocity)[r * OUT + o] = __float2bfloat16_rn(v);
+      else reinterpret_cast<float*>(velocity)[r * OUT + o] = v;
+    }
   }
 }
 
@@ -393,7 +498,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnParams p) {
     for (int i = 0; i < DPL; ++i) o[i] = o[i] * corr + pe * v[i];
     m = mn;
   }
-  const float inv = 1.f / l;
+  const float inv = l > 0.f ? 1.f / l : 0.f;  // no valid key (text-only sequence, all padded): zeros
   T* out = reinterpret_cast<T*>(p.out);
 #pragma unroll
   for (int i = 0; i < DPL; ++i) {
@@ -402,6 +507,35 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnParams p) {
     if constexpr (sizeof(T) == 2) out[row * HD + (long)h * D + d0 + i] = __float2bfloat16_rn(y);
     else out[row * HD + (long)h * D + d0 + i] = y;
   }
+}
+
+// ----------------------------------------------------------------------------- sampler step
+// v = v_cond + g (v_cond - v_uncond); x += (sigma_next - sigma) v; then the next model input
+// (x repeated `copies` times) and its timestep sigma_next.
+template <bool BF16>
+__global__ void euler_cfg_kernel(long long n, float* __restrict__ x, const void* __restrict__ vc,
+                                 const void* __restrict__ vu, float g, float dsigma, void* __restrict__ xm,
+                                 int copies, float* __restrict__ t_out, float sigma_next) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    float c = 0.f, u = 0.f;  // no v_cond: v = 0 (only copies x into the model input)
+    if (BF16) {
+      if (vc) c = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vc)[i]);
+      if (vu) u = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(vu)[i]);
+    } else {
+      if (vc) c = reinterpret_cast<const float*>(vc)[i];
+      if (vu) u = reinterpret_cast<const float*>(vu)[i];
+    }
+    const float v = vu ? c + g * (c - u) : c;
+    const float y = x[i] + dsigma * v;
+    x[i] = y;
+    if (xm) {
+      for (int k = 0; k < copies; ++k) {
+        if (BF16) reinterpret_cast<__nv_bfloat16*>(xm)[k * n + i] = __float2bfloat16_rn(y);
+        else reinterpret_cast<float*>(xm)[k * n + i] = y;
+      }
+    }
+  }
+  if (t_out && blockIdx.x == 0 && threadIdx.x < copies) t_out[threadIdx.x] = sigma_next;
 }
 
 inline int check_launch(const char* what) {
@@ -430,6 +564,39 @@ int launch_rope_tables(const float* pos, int S, int a0, int a1, int a2, float th
 int launch_modulation(const float* temb, const float* table, int B, int C, float* mod, cudaStream_t stream) {
   modulation_kernel<<<grid_for((long)B * 6 * C, 256), 256, 0, stream>>>(temb, table, B, C, mod);
   return check_launch("modulation");
+}
+
+int launch_unit_modulation(int B, int C, float* mod, cudaStream_t stream) {
+  unit_modulation_kernel<<<grid_for((long)B * 6 * C, 256), 256, 0, stream>>>(B, C, mod);
+  return check_launch("unit_modulation");
+}
+
+int launch_identity_rope(long n, float* cs, float* sn, cudaStream_t stream) {
+  if (n <= 0) return KREA2_OK;
+  identity_rope_kernel<<<grid_for(n, 256), 256, 0, stream>>>(n, cs, sn);
+  return check_launch("identity_rope");
+}
+
+int launch_layer_projection(const float* x, const float* w, long rows, int L, int C, void* out, bool out_bf16,
+                            cudaStream_t stream) {
+  if (rows <= 0) return KREA2_OK;
+  if (out_bf16) layer_projection_kernel<true><<<grid_for(rows * C, 256), 256, 0, stream>>>(x, w, rows, L, C, out);
+  else layer_projection_kernel<false><<<grid_for(rows * C, 256), 256, 0, stream>>>(x, w, rows, L, C, out);
+  return check_launch("layer_projection");
+}
+
+int launch_to_f32(const void* in, bool in_bf16, long n, float* out, cudaStream_t stream) {
+  if (n <= 0) return KREA2_OK;
+  if (in_bf16) to_f32_kernel<true><<<grid_for(n, 256), 256, 0, stream>>>(in, n, out);
+  else to_f32_kernel<false><<<grid_for(n, 256), 256, 0, stream>>>(in, n, out);
+  return check_launch("to_f32");
+}
+
+int launch_to_dtype(const float* in, long n, void* out, bool out_bf16, cudaStream_t stream) {
+  if (n <= 0) return KREA2_OK;
+  if (out_bf16) from_f32_kernel<true><<<grid_for(n, 256), 256, 0, stream>>>(in, n, out);
+  else from_f32_kernel<false><<<grid_for(n, 256), 256, 0, stream>>>(in, n, out);
+  return check_launch("to_dtype");
 }
 
 int launch_mod_rmsnorm(const float* h, const float* w, const float* temb, const float* table, int chunk, int B, int S,
@@ -467,20 +634,27 @@ int launch_time_embed(const Krea2Dims* d, int B, bool w_bf16, const float* t, co
 }
 
 int launch_final_layer(const Krea2Dims* d, int B, int T, int N, bool bf16, const float* h, const float* e,
-                       const Krea2ModelWeights* w, float* ybuf, void* velocity, cudaStream_t stream) {
-  const int S = T + N, C = d->C;
-  if ((long)B * N == 0) return KREA2_OK;
-  final_norm_kernel<<<(unsigned)((long)B * N), 256, 0, stream>>>(h, e, w->final_norm_w, w->final_table, T, N, S, C,
-                                                                  d->eps, ybuf);
-  int rc = check_launch("final_norm");
-  if (rc) return rc;
-  SimtGemmParams p{};
-  p.M = B * N;
-  p.N = d->in_ch;
-  p.K = C;
-  p.out = velocity;
-  p.bias = w->final_b;
-  return gemm_simt(bf16 ? SEPI_BIAS_BF16 : SEPI_BIAS_F32, p, ybuf, false, w->final_w, bf16, stream);
+                       const Krea2ModelWeights* w, void* velocity, cudaStream_t stream) {
+  const long rows = (long)B * N;
+  if (rows == 0) return KREA2_OK;
+  if (d->in_ch > FL_MAX_OUT) return set_error(KREA2_ERR_UNSUPPORTED, "in_channels must be <= %d", FL_MAX_OUT);
+  const unsigned grid = (unsigned)((rows + FL_ROWS - 1) / FL_ROWS);
+  if (bf16)
+    final_layer_kernel<true><<<grid, 256, 0, stream>>>(h, e, w->final_norm_w, w->final_table, w->final_w, w->final_b,
+                                                        B, T, N, d->C, d->in_ch, d->eps, velocity);
+  else
+    final_layer_kernel<false><<<grid, 256, 0, stream>>>(h, e, w->final_norm_w, w->final_table, w->final_w, w->final_b,
+                                                         B, T, N, d->C, d->in_ch, d->eps, velocity);
+  return check_launch("final_layer");
+}
+
+int launch_euler_cfg(bool bf16, long long n, float* x, const void* vc, const void* vu, float g, float sigma,
+                     float sigma_next, void* xm, int copies, float* t_out, cudaStream_t stream) {
+  if (n <= 0) return KREA2_OK;
+  const float ds = sigma_next - sigma;
+  if (bf16) euler_cfg_kernel<true><<<grid_for(n, 256), 256, 0, stream>>>(n, x, vc, vu, g, ds, xm, copies, t_out, sigma_next);
+  else euler_cfg_kernel<false><<<grid_for(n, 256), 256, 0, stream>>>(n, x, vc, vu, g, ds, xm, copies, t_out, sigma_next);
+  return check_launch("euler_cfg");
 }
 
 int launch_copy_text_rows(const void* text, bool bf16, int B, int T, int S, int C, float* h, cudaStream_t stream) {

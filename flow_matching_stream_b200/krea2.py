@@ -19,7 +19,9 @@ from ._lib import KREA2_BF16, KREA2_F32, KREA2_EPI_RESID, KREA2_EPI_STORE, KREA2
 
 __all__ = [
     "Krea2Error", "lib", "dims_struct", "dtype_code", "workspace_size", "attention_workspace_size",
-    "rope_tables", "gqa_attention", "gqa_attention_noalloc", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
+    "rope_tables", "gqa_attention", "gqa_attention_noalloc", "block_causal_key_end", "gqa_attention_block_causal", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
+    "text_dims_struct", "TextWeights", "text_fusion_workspace_size", "text_fusion",
+    "shift_mu", "sigma_schedule", "euler_cfg_step", "sample_workspace_size", "sample",
     "block_forward", "block_forward_traced", "BLOCK_STEPS", "launch_count", "backbone_forward", "check_device_error", "BlockWeights", "ModelWeights",
     "interleave_gate_up", "KREA2_BF16", "KREA2_F32", "KREA2_EPI_STORE", "KREA2_EPI_SWIGLU", "KREA2_EPI_RESID",
 ]
@@ -129,6 +131,26 @@ def gqa_attention_noalloc(dims, B: int, T: int, N: int, qkvg: torch.Tensor, q_no
                                              _p(text_mask), _p(out), _s(stream)))
 
 
+def block_causal_key_end(image_ids: np.ndarray) -> np.ndarray:
+    """Per-query key prefix of the block-causal pattern (host computation in the library)."""
+    ids = np.ascontiguousarray(image_ids, dtype=np.int32)
+    out = np.zeros(len(ids), dtype=np.int32)
+    _check(lib().krea2_block_causal_key_end(ids.ctypes.data, len(ids), out.ctypes.data))
+    return out
+
+
+def gqa_attention_block_causal(dims, B: int, T: int, N: int, qkvg: torch.Tensor, q_norm_w: torch.Tensor,
+                               k_norm_w: torch.Tensor, cos: torch.Tensor, sin: torch.Tensor,
+                               text_mask: Optional[torch.Tensor], key_end: torch.Tensor, out: torch.Tensor,
+                               workspace: torch.Tensor, stream=None) -> None:
+    _want(key_end, torch.int32, "key_end")
+    _want(out, qkvg.dtype, "out")
+    _check(lib().krea2_gqa_attention_block_causal(
+        ctypes.byref(dims_struct(dims)), B, T, N, dtype_code(qkvg.dtype), _p(qkvg), _p(q_norm_w), _p(k_norm_w),
+        _p(cos), _p(sin), _p(text_mask), _p(key_end), _p(out), _p(workspace),
+        workspace.numel() * workspace.element_size(), _s(stream)))
+
+
 def modulated_rmsnorm(dims, B: int, S: int, h: torch.Tensor, norm_w: torch.Tensor, temb: torch.Tensor,
                       table: torch.Tensor, chunk: int, out: torch.Tensor, stream=None) -> None:
     _check(lib().krea2_modulated_rmsnorm(ctypes.byref(dims_struct(dims)), B, S, dtype_code(out.dtype), _p(h),
@@ -153,9 +175,9 @@ def time_embed(dims, timestep: torch.Tensor, mw: "ModelWeights", temb_out: torch
 
 
 def final_layer(dims, B: int, T: int, N: int, h: torch.Tensor, e: torch.Tensor, mw: "ModelWeights",
-                velocity: torch.Tensor, scratch: torch.Tensor, stream=None) -> None:
+                velocity: torch.Tensor, stream=None) -> None:
     _check(lib().krea2_final_layer(ctypes.byref(dims_struct(dims)), B, T, N, mw.dtype_code, _p(h), _p(e),
-                                   ctypes.byref(mw.struct), _p(velocity), _p(scratch), _s(stream)))
+                                   ctypes.byref(mw.struct), _p(velocity), _s(stream)))
 
 
 def block_forward(dims, B: int, T: int, N: int, h: torch.Tensor, temb: torch.Tensor, bw: "BlockWeights",
@@ -165,6 +187,62 @@ def block_forward(dims, B: int, T: int, N: int, h: torch.Tensor, temb: torch.Ten
     _check(lib().krea2_block_forward(ctypes.byref(dims_struct(dims)), B, T, N, bw.dtype_code, _p(h), _p(temb),
                                      ctypes.byref(bw.struct), _p(cos), _p(sin), _p(text_mask), _p(workspace),
                                      workspace.numel() * workspace.element_size(), _s(stream)))
+
+
+def text_dims_struct(td) -> _lib.Krea2TextDims:
+    s = _lib.Krea2TextDims()
+    for f in ("Dt", "L", "H", "Hkv", "D", "F", "n_layerwise", "n_refiner", "C"):
+        setattr(s, f, getattr(td, f))
+    s.eps = float(td.eps)
+    return s
+
+
+def text_fusion_workspace_size(td, B: int, T: int, dtype: torch.dtype) -> int:
+    return int(lib().krea2_text_fusion_workspace_size(ctypes.byref(text_dims_struct(td)), B, T, dtype_code(dtype)))
+
+
+def text_fusion(td, B: int, T: int, ehs: torch.Tensor, text_mask: Optional[torch.Tensor], tw: "TextWeights",
+                text_out: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    _want(ehs, tw.dtype, "ehs")
+    _want(text_out, tw.dtype, "text_out")
+    _check(lib().krea2_text_fusion(ctypes.byref(text_dims_struct(td)), B, T, tw.dtype_code, _p(ehs), _p(text_mask),
+                                   ctypes.byref(tw.struct), _p(text_out), _p(workspace),
+                                   workspace.numel() * workspace.element_size(), _s(stream)))
+
+
+def shift_mu(image_seq_len: int) -> float:
+    return float(lib().krea2_shift_mu(image_seq_len))
+
+
+def sigma_schedule(n_steps: int, mu: float) -> np.ndarray:
+    out = np.zeros(n_steps + 1, dtype=np.float32)
+    _check(lib().krea2_sigma_schedule(n_steps, mu, out.ctypes.data))
+    return out
+
+
+def euler_cfg_step(x: torch.Tensor, v_cond: torch.Tensor, v_uncond: Optional[torch.Tensor], guidance: float,
+                   sigma: float, sigma_next: float, x_model: Optional[torch.Tensor] = None, copies: int = 1,
+                   timestep_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    _want(x, torch.float32, "x")
+    _check(lib().krea2_euler_cfg_step(dtype_code(v_cond.dtype), x.numel(), _p(x), _p(v_cond), _p(v_uncond),
+                                      guidance, sigma, sigma_next, _p(x_model), copies, _p(timestep_out),
+                                      _s(stream)))
+
+
+def sample_workspace_size(dims, T: int, N: int, dtype: torch.dtype, cfg: bool) -> int:
+    return int(lib().krea2_sample_workspace_size(ctypes.byref(dims_struct(dims)), T, N, dtype_code(dtype), int(cfg)))
+
+
+def sample(dims, T: int, N: int, latents: torch.Tensor, text_cond: torch.Tensor, text_uncond: Optional[torch.Tensor],
+           mask_cond: Optional[torch.Tensor], mask_uncond: Optional[torch.Tensor], position_ids: torch.Tensor,
+           sigmas: np.ndarray, guidance: float, mw: "ModelWeights", workspace: torch.Tensor, stream=None) -> None:
+    """The device sampling loop (krea2_sample); `sigmas` is a host array of n_steps + 1 values."""
+    _want(latents, torch.float32, "latents")
+    sg = np.ascontiguousarray(sigmas, dtype=np.float32)
+    _check(lib().krea2_sample(ctypes.byref(dims_struct(dims)), T, N, mw.dtype_code, _p(latents), _p(text_cond),
+                              _p(text_uncond), _p(mask_cond), _p(mask_uncond), _p(position_ids), sg.ctypes.data,
+                              len(sg) - 1, guidance, ctypes.byref(mw.struct), _p(workspace),
+                              workspace.numel() * workspace.element_size(), _s(stream)))
 
 
 BLOCK_STEPS = ("modulation", "norm1", "qkv_proj", "attention", "out_proj_resid", "norm2", "gate_up_swiglu",
@@ -256,6 +334,33 @@ class BlockWeights:
              "norm1_w": n((C,), 0.1).float(), "norm2_w": n((C,), 0.1).float(), "q_norm_w": n((D,), 0.1).float(),
              "k_norm_w": n((D,), 0.1).float(), "table": n((6, C), 0.1).float()}
         return BlockWeights(w, dtype, device)
+
+
+class TextWeights:
+    """Text-fusion device tensors: layerwise / refiner blocks (no modulation table), the layer-axis
+    projection and txt_in."""
+
+    def __init__(self, tw: Dict[str, object], dtype: torch.dtype, device):
+        self.dtype = dtype
+        self.dtype_code = dtype_code(dtype)
+        self.layerwise = [BlockWeights(dict(w, table=np.zeros((6, 1), np.float32)), dtype, device)
+                          for w in tw["layerwise"]]
+        self.refiner = [BlockWeights(dict(w, table=np.zeros((6, 1), np.float32)), dtype, device)
+                        for w in tw["refiner"]]
+        self.layer_w = _dev(tw["layer_w"], torch.float32, device)
+        self.txt_in_w = _dev(tw["txt_in_w"], dtype, device)
+        self.txt_in_b = _dev(tw["txt_in_b"], torch.float32, device)
+        self._lw = (_lib.Krea2BlockWeights * max(1, len(self.layerwise)))()
+        self._rf = (_lib.Krea2BlockWeights * max(1, len(self.refiner)))()
+        for arr, blocks in ((self._lw, self.layerwise), (self._rf, self.refiner)):
+            for i, b in enumerate(blocks):
+                b.fill(arr[i])
+                arr[i].scale_shift_table = None   # fusion blocks carry no time modulation
+        s = _lib.Krea2TextWeights()
+        s.layerwise = ctypes.cast(self._lw, ctypes.POINTER(_lib.Krea2BlockWeights))
+        s.refiner = ctypes.cast(self._rf, ctypes.POINTER(_lib.Krea2BlockWeights))
+        s.layer_w, s.txt_in_w, s.txt_in_b = _p(self.layer_w), _p(self.txt_in_w), _p(self.txt_in_b)
+        self.struct = s
 
 
 class ModelWeights:

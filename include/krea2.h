@@ -174,6 +174,26 @@ int krea2_gqa_attention_noalloc(const Krea2Dims* dims, int B, int T, int N, int 
                                 const float* cos, const float* sin, const uint8_t* text_mask,
                                 void* out, void* stream);
 
+/* Block-causal attention (page "QwenImage21Transformer2DModel": query q reads key k iff
+ * q >= k or both lie in the same image block; a variant for models built on this block).
+ * That pattern is a per-query key prefix: q reads keys [0, key_end[q]) with key_end[q] = q + 1
+ * for a text token and the end of its image block for an image token.
+ * krea2_block_causal_key_end computes key_end (HOST arrays, S entries) from image_ids (-1 at text
+ * positions, one id per image block, blocks contiguous). Returns KREA2_ERR_ARG if a block is not
+ * contiguous. */
+int krea2_block_causal_key_end(const int32_t* image_ids, int S, int32_t* key_end);
+
+/* krea2_gqa_attention under the block-causal pattern: key_end (S) int32 DEVICE array from
+ * krea2_block_causal_key_end, shared by all batch rows; the text mask still removes padded keys.
+ * A query with no readable key outputs zeros. Tensor-core path only (bf16, D = 128,
+ * H/Hkv in {1, 2, 4}); other shapes return KREA2_ERR_UNSUPPORTED. Workspace as
+ * krea2_gqa_attention. Key tiles beyond every query of a CTA are never loaded. */
+int krea2_gqa_attention_block_causal(const Krea2Dims* dims, int B, int T, int N, int dtype,
+                                     const void* qkvg, const float* q_norm_w, const float* k_norm_w,
+                                     const float* cos, const float* sin, const uint8_t* text_mask,
+                                     const int32_t* key_end, void* out, void* workspace,
+                                     size_t ws_bytes, void* stream);
+
 /* Shared modulation of one block plus its table, then a modulated RMSNorm ([ARCH] §四.2,
  * §四.4): with mod = temb (B, 6C) viewed as (B, 6, C) plus table (6, C),
  *   out[b, s] = (1 + mod[b, chunk]) * rms(h[b, s]) * (1 + norm_w) + mod[b, chunk + 1].
@@ -209,11 +229,10 @@ int krea2_time_embed(const Krea2Dims* dims, int B, int dtype, const float* times
 /* Final layer on image rows ([ARCH] §四.6): (scale, shift) = final_table + e;
  * y = (1 + scale) * rms(x) * (1 + final_norm_w) + shift; velocity = y · final_wᵀ + final_b.
  * h (B*S, C) fp32 full sequence (text rows are skipped, [ARCH] §二); e (B, C) fp32;
- * velocity (B, N, in_ch) in `dtype`; scratch: device fp32 buffer of >= B*N*C floats
- * (holds y). Reads w->final_*. */
+ * velocity (B, N, in_ch) in `dtype` (in_ch <= 64). Reads w->final_*. One fused kernel. */
 int krea2_final_layer(const Krea2Dims* dims, int B, int T, int N, int dtype,
                       const float* h, const float* e, const Krea2ModelWeights* w,
-                      void* velocity, float* scratch, void* stream);
+                      void* velocity, void* stream);
 
 /* One Krea2TransformerBlock forward ([ARCH] §四.2), in place on the fp32 residual:
  *   mod = temb + table;  xn = (1+prescale)*norm1(h) + preshift;
@@ -238,6 +257,80 @@ int krea2_block_forward_traced(const Krea2Dims* dims, int B, int T, int N, int d
 
 /* Number of kernels this library has launched in this process so far (all entry points). */
 unsigned long long krea2_launch_count(void);
+
+/* ---- sampler (the steps either side of the backbone in [PIPE] __call__) ----------------------
+ * Resolution-aware shift of the sigma schedule ([PIPE] scheduler: use_dynamic_shifting with
+ * base_shift 0.5, max_shift 1.15, base_image_seq_len 256, max_image_seq_len 6400): mu on the
+ * straight line through (256, 0.5) and (6400, 1.15) in image_seq_len (a reading; the distilled
+ * checkpoint uses the fixed mu = 1.15). Host function. */
+double krea2_shift_mu(int image_seq_len);
+
+/* Sigma schedule ([PIPE] __call__: default grid linspace(1, 1/n_steps, n_steps), exponential time
+ * shift sigma' = e^mu / (e^mu + (1/sigma - 1)) (a reading), then the terminal 0). Writes n_steps + 1
+ * values to sigmas_out (HOST memory), computed in fp64. KREA2_ERR_ARG for n_steps < 1. */
+int krea2_sigma_schedule(int n_steps, double mu, float* sigmas_out);
+
+/* One sampler step on the device ([PIPE] guidance_scale, scheduler step; [ARCH] §五):
+ *   v = v_cond + guidance * (v_cond - v_uncond)   (v_uncond NULL or guidance <= 0: v = v_cond),
+ *   x <- x + (sigma_next - sigma) * v.
+ * x (n) fp32 latents, updated in place; v_cond, v_uncond (n) in `dtype`;
+ * x_model (copies * n) in `dtype`, optional: receives `copies` back-to-back copies of the new x
+ * (the next model input, copies = 2 for a [cond, uncond] batch); timestep_out (copies) fp32,
+ * optional: receives sigma_next (the next model timestep, t / num_train_timesteps). */
+int krea2_euler_cfg_step(int dtype, long long n, float* x, const void* v_cond, const void* v_uncond,
+                         float guidance, float sigma, float sigma_next, void* x_model, int copies,
+                         float* timestep_out, void* stream);
+
+/* Bytes of device workspace krea2_sample needs (0 on invalid arguments). */
+size_t krea2_sample_workspace_size(const Krea2Dims* dims, int T, int N, int dtype, int cfg);
+
+/* The whole sampling loop on the device, for one image ([PIPE] __call__): for i = 0..n_steps-1 the
+ * backbone runs at timestep sigmas[i] on the batch [cond] (guidance <= 0) or [cond, uncond]
+ * (guidance > 0, one batch-2 forward), then krea2_euler_cfg_step moves the latents to
+ * sigmas[i+1]. latents (N, in_ch) fp32, in/out (initial noise in, sample out); text_cond,
+ * text_uncond (T, C) in `dtype` (text_uncond unused when guidance <= 0); mask_cond, mask_uncond
+ * (T) uint8 or NULL; position_ids (T+N, 3); sigmas: HOST array of n_steps + 1 values (e.g. from
+ * krea2_sigma_schedule); workspace >= krea2_sample_workspace_size(dims, T, N, dtype, guidance > 0).
+ * Asynchronous; every launch goes to `stream`, so the call can be captured in a CUDA graph. */
+int krea2_sample(const Krea2Dims* dims, int T, int N, int dtype, float* latents,
+                 const void* text_cond, const void* text_uncond, const uint8_t* mask_cond,
+                 const uint8_t* mask_uncond, const float* position_ids, const float* sigmas,
+                 int n_steps, float guidance, const Krea2ModelWeights* w, void* workspace,
+                 size_t ws_bytes, void* stream);
+
+/* ---- text conditioning (Krea2TextFusion + txt_in, [ARCH] §四.1 and §四 module list) ----------
+ * Text-fusion hyper-parameters ([API] text_hidden_dim Dt = 2560, num_text_layers L = 12,
+ * text_num_attention_heads H = 20, text_num_key_value_heads Hkv = 20, text_intermediate_size
+ * F = 6912, num_layerwise_text_blocks 2, num_refiner_text_blocks 2; D = Dt / H head dim; C the
+ * backbone hidden size that txt_in projects to). */
+typedef struct {
+  int Dt, L, H, Hkv, D, F, n_layerwise, n_refiner, C;
+  float eps;
+} Krea2TextDims;
+
+/* Text-fusion parameters. layerwise / refiner: HOST arrays of n_layerwise / n_refiner block
+ * weights (Krea2BlockWeights with hidden size Dt; scale_shift_table must be NULL: the fusion
+ * blocks have no time modulation); layer_w (L) fp32: Linear(L, 1, bias=False) over the layer
+ * axis; txt_in_w (C, Dt) in `dtype`, txt_in_b (C) fp32 (a reading: txt_in is Linear + bias). */
+typedef struct {
+  const Krea2BlockWeights* layerwise;
+  const Krea2BlockWeights* refiner;
+  const float* layer_w;
+  const void* txt_in_w;
+  const float* txt_in_b;
+} Krea2TextWeights;
+
+size_t krea2_text_fusion_workspace_size(const Krea2TextDims* td, int B, int T, int dtype);
+
+/* Text conditioning from the stacked encoder states ([ARCH] §四.1): each token's (L, Dt) stack is
+ * its own sequence through the layerwise blocks (pre-norm blocks with q/k RMSNorm, sigmoid-gated
+ * MHA and SwiGLU, no RoPE, no time modulation: a reading); Linear(L, 1) collapses the layer axis;
+ * the token sequence goes through the refiner blocks under the text mask; txt_in projects to C.
+ * ehs (B, T, L, Dt) in `dtype`; text_mask (B, T) uint8 or NULL; text_out (B, T, C) in `dtype`,
+ * ready for krea2_backbone_forward's text_states. Computed once per prompt (no timestep). */
+int krea2_text_fusion(const Krea2TextDims* td, int B, int T, int dtype, const void* ehs,
+                      const uint8_t* text_mask, const Krea2TextWeights* w, void* text_out,
+                      void* workspace, size_t ws_bytes, void* stream);
 
 /* Backbone forward from post-fusion text features ([API] forward; [ARCH] §四 data flow):
  * RoPE tables; time path; x = cat([text_states, img_in(hidden_states)]); n_layers blocks;

@@ -448,3 +448,52 @@ def txt_in(x: np.ndarray, w: np.ndarray, b: np.ndarray, dtype=np.float64) -> np.
     """Krea2TextProjection ([ARCH] §四 module list: txt_in(text_hidden_dim -> hidden_size)).
     READING: its internals are not given; a plain Linear(Dt, C) with bias."""
     return x.astype(dtype) @ w.astype(dtype).T + b.astype(dtype)
+
+
+# ----------------------------------------------------------------------------- block-causal variant
+
+def image_block_ids(segments: Sequence[Tuple[str, int]]) -> np.ndarray:
+    """Token metadata of the block-causal variant (page "QwenImage21Transformer2DModel",
+    build_token_metadata): the joint sequence as ("text", n) / ("image", n) segments in order;
+    -1 at text positions and one id per image block. Block boundaries come from the segment
+    sizes, so two adjacent image segments stay two blocks."""
+    ids = []
+    nxt = 0
+    for kind, n in segments:
+        if kind == "text":
+            ids += [-1] * n
+        else:
+            ids += [nxt] * n
+            nxt += 1
+    return np.asarray(ids, dtype=np.int64)
+
+
+def block_causal_allowed(ids: np.ndarray) -> np.ndarray:
+    """Attention pattern of the QwenImage 2.1 page: query q may read key k iff
+    (q_idx >= kv_idx) or (q and k lie in the same image block). Returns (S, S) bool."""
+    S = len(ids)
+    q = np.arange(S)[:, None]
+    k = np.arange(S)[None, :]
+    same = (ids[:, None] == ids[None, :]) & (ids[:, None] >= 0)
+    return (q >= k) | same
+
+
+def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.ndarray, key_valid: np.ndarray,
+                     scale: float) -> np.ndarray:
+    """GQA softmax attention where query row i of batch row b reads keys with
+    allowed[i, j] and key_valid[b, j]; a row with no readable key outputs zeros.
+    q (B, S, H, D); k, v (B, S, Hkv, D); allowed (S, S); key_valid (B, S). Returns fp64."""
+    B, S, H, D = q.shape
+    G = H // k.shape[2]
+    out = np.zeros((B, S, H, D), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            j = h // G
+            for i in range(S):
+                idx = np.nonzero(allowed[i] & key_valid[b])[0]
+                if idx.size == 0:
+                    continue
+                s = (k[b, idx, j, :] @ q[b, i, h, :]).astype(np.float64) * scale
+                p = np.exp(s - s.max())
+                out[b, i, h, :] = (p / p.sum()) @ v[b, idx, j, :].astype(np.float64)
+    return out

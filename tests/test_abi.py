@@ -1,6 +1,8 @@
 """The C-ABI library loads without a GPU, exports every entry point of include/krea2.h, and
 rejects bad arguments on the host before anything is launched."""
 import ctypes
+
+import numpy as np
 import os
 import re
 
@@ -68,3 +70,33 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         _lib.load()
+
+
+def test_sigma_schedule_host_functions_match_oracle(K2):
+    # host-side schedule of the library (C code) against the oracle's fp64 schedule
+    from oracle import krea2_oracle as O
+    for n in (28, 8, 1):
+        for mu in (O.shift_mu(4096), 1.15, 0.0):
+            got = K2.sigma_schedule(n, mu)
+            ref = O.shifted_sigmas(n, mu)
+            assert got.shape == ref.shape
+            assert abs(float(got[-1])) == 0.0 and abs(float(got[0]) - 1.0) < 1e-7
+            assert float(np.max(np.abs(got - ref))) < 1e-7
+    for L in (256, 1024, 4096, 6400):
+        assert abs(K2.shift_mu(L) - O.shift_mu(L)) < 1e-12
+    assert K2.lib().krea2_sigma_schedule(0, 0.5, None) == -1
+
+
+def test_block_causal_key_end_matches_the_oracle_pattern(K2):
+    from oracle import krea2_oracle as O
+    rng = np.random.default_rng(5)
+    for _ in range(30):
+        segs = [(("text", "image")[rng.integers(2)], int(rng.integers(1, 9))) for _ in range(rng.integers(1, 8))]
+        ids = O.image_block_ids(segs)
+        kend = K2.block_causal_key_end(ids)
+        allowed = O.block_causal_allowed(ids)
+        S = len(ids)
+        assert all(allowed[q].tolist() == [k < kend[q] for k in range(S)] for q in range(S))
+    bad = np.array([0, 0, -1, 0], dtype=np.int32)  # block 0 split in two runs
+    with pytest.raises(K2.Krea2Error):
+        K2.block_causal_key_end(bad)

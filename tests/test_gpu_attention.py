@@ -109,3 +109,56 @@ def test_attention_sweep_sampled_rows(K2, grid):
     rows = sample_rows(wl.T, wl.S)
     ref = oracle_attention(d, x, w, pos, wl.B, wl.T, wl.N, mask, rows=rows, dtype=np.float32)
     assert rel_err(out[:, rows], ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("H,Hkv", [(8, 8), (8, 4), (20, 20)])
+def test_attention_bf16_other_group_sizes(K2, H, Hkv):
+    # tensor-core path with 1 or 2 query heads per KV head (128 or 64 positions per tile)
+    d = KI.Dims(C=H * 128, H=H, Hkv=Hkv, D=128, F=1024, axes=(32, 48, 48))
+    B, T, gh, gw = 2, 70, 9, 11
+    mask = KI.mask_from_lengths(T, [70, 17])
+    x, w, pos, out = run_attention(K2, d, B, T, gh, gw, mask, torch.bfloat16)
+    ref = oracle_attention(d, x, w, pos, B, T, gh * gw, mask)
+    assert rel_err(out, ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("segs,lengths", [
+    ([("text", 150), ("image", 64), ("text", 30), ("image", 400)], [244, 100]),   # ragged, padded text
+    ([("text", 40), ("image", 130), ("image", 70)], [40, 40]),                   # adjacent image blocks
+    ([("text", 200)], [200, 1]),                                                  # pure causal text
+])
+def test_attention_block_causal(K2, segs, lengths):
+    d = KI.FULL
+    ids = O.image_block_ids(segs)
+    S = len(ids)
+    B = 2
+    T = S  # the whole sequence takes the text mask (image positions marked valid)
+    mask = KI.mask_from_lengths(T, lengths)
+    for b in range(B):
+        mask[b, ids >= 0] = True
+    x = KI.qkvg_raw(d, B, S)
+    w = KI.block_weights(d, 0)
+    pos = np.zeros((S, 3), dtype=np.float32)
+    pos[:, 1] = np.arange(S) // 16
+    pos[:, 2] = np.arange(S) % 16
+    cs = torch.empty(S, 64, device="cuda")
+    sn = torch.empty_like(cs)
+    K2.rope_tables(d, dev(pos, torch.float32), cs, sn)
+    kend = dev(K2.block_causal_key_end(ids), torch.int32)
+    out = torch.empty(B * S, d.HD, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(K2.attention_workspace_size(d, B, T - 1, 1, torch.bfloat16), dtype=torch.uint8, device="cuda")
+    # the whole sequence sits under the text mask (T = S, no separate image tokens)
+    K2.gqa_attention_block_causal(d, B, T, 0, dev(x, torch.bfloat16), dev(w["q_norm_w"], torch.float32),
+                                  dev(w["k_norm_w"], torch.float32), cs, sn, dev(mask.astype(np.uint8), torch.uint8),
+                                  kend, out, ws)
+    K2.check_device_error()
+    c, s = O.rope_cos_sin(pos, d.axes, d.theta)
+    xf = x.astype(np.float64).reshape(B, S, -1)
+    q = O.apply_rope(O.rms_norm(xf[..., :d.HD].reshape(B, S, d.H, d.D), w["q_norm_w"], d.eps), c, s)
+    k = O.apply_rope(O.rms_norm(xf[..., d.HD:d.HD + d.KVD].reshape(B, S, d.Hkv, d.D), w["k_norm_w"], d.eps), c, s)
+    v = xf[..., d.HD + d.KVD:d.HD + 2 * d.KVD].reshape(B, S, d.Hkv, d.D)
+    g = xf[..., d.HD + 2 * d.KVD:]
+    kv = mask
+    o = O.masked_attention(q, k, v, O.block_causal_allowed(ids), kv, 1.0 / np.sqrt(d.D))
+    ref = o.reshape(B, S, d.HD) * O.sigmoid(g)
+    assert rel_err(host(out).reshape(B, S, d.HD), ref) < TOL_BF16

@@ -116,8 +116,6 @@ def test_final_layer(K2, dims, dtype, tol):
     h = KI.residual(dims, B, S)
     e = KI.temb(dims, B)[:, :dims.C]
     vel = torch.empty(B * N, dims.in_ch, device="cuda", dtype=dtype)
-    scratch = torch.empty(B * N, dims.C, device="cuda")
-    K2.final_layer(dims, B, T, N, dev(h.reshape(B * S, dims.C), torch.float32), dev(e, torch.float32), mw, vel,
-                   scratch)
+    K2.final_layer(dims, B, T, N, dev(h.reshape(B * S, dims.C), torch.float32), dev(e, torch.float32), mw, vel)
     ref = O.final_layer(h[:, T:], e, mw_h, dims.eps)
     assert rel_err(host(vel).reshape(B, N, dims.in_ch), ref) < tol

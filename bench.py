@@ -319,6 +319,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
 
     sampler = time_sampler(K2, torch, d, mw, dev)
     text = time_text_fusion(K2, torch, dev, args.steps)
+    sweep = time_attention_sweep(K2, torch, dev, args.steps, pk)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -333,6 +334,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         "backbone_ms_per_step": ms_step,
         "sampler_1024sq": sampler,
         "text_fusion_once_per_prompt": text,
+        "attention_sweep": sweep,
         "pct_of_tensor_peak": {"burst": value / world / pk["bf16_tflops"],
                                "sustained": value / world / pk["bf16_tflops_sustained"]},
         "block_1024sq_cfg": cfg_res,
@@ -444,6 +446,44 @@ def time_text_fusion(K2, torch, dev, steps: int) -> dict:
     per_row = 2 * bd.C * (bd.qkvg_cols + bd.HD + 2 * bd.F + bd.F)
     fl = per_row * (td.n_layerwise * B * T * td.L + td.n_refiner * B * T) + 2 * B * T * td.Dt * td.C
     return {"workload": "text_fusion_2x512x12x2560", "ms": ms, "gemm_tflops": fl / (ms / 1e3) / 1e12}
+
+
+def time_attention_sweep(K2, torch, dev, steps: int, pk: dict) -> list:
+    """The attention-only sweep: 48 q / 12 kv heads x 128 with 512 text tokens (random valid
+    length) and 32^2 .. 128^2 image grids, through krea2_gqa_attention (q/k norm + RoPE pass and
+    the flash-attention kernel). FLOPs count valid keys only."""
+    out = []
+    for grid in (32, 64, 96, 128):
+        wl = KI.attn_sweep(grid)
+        d = wl.dims
+        B, T, N, S = wl.B, wl.T, wl.N, wl.S
+        g = torch.Generator(device=dev).manual_seed(grid)
+        x = torch.randn(B * S, d.qkvg_cols, device=dev, generator=g).to(torch.bfloat16)
+        qw = torch.randn(d.D, device=dev, generator=g) * 0.1
+        kw = torch.randn(d.D, device=dev, generator=g) * 0.1
+        cs = torch.empty(S, d.D // 2, device=dev)
+        sn = torch.empty_like(cs)
+        K2.rope_tables(d, torch.from_numpy(wl.positions()).to(dev), cs, sn)
+        mask = torch.from_numpy(wl.mask().astype(np.uint8)).to(dev)
+        o = torch.empty(B * S, d.HD, device=dev, dtype=torch.bfloat16)
+        ws = torch.empty(K2.attention_workspace_size(d, B, T, N, torch.bfloat16), dtype=torch.uint8, device=dev)
+        run = lambda: K2.gqa_attention(d, B, T, N, x, qw, kw, cs, sn, mask, o, ws)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        K2.check_device_error()
+        ms = e0.elapsed_time(e1) / steps
+        fl = 4.0 * d.D * d.H * S * (wl.lengths[0] + N)
+        out.append({"grid": grid, "tokens": S, "valid_text": wl.lengths[0], "ms": ms,
+                    "tflops": fl / (ms / 1e3) / 1e12, "frac_burst": fl / (ms / 1e3) / 1e12 / pk["bf16_tflops"]})
+        del x, o, ws
+    return out
 
 
 def traced_block_kernels(K2, torch, d, B, T, N, lengths, bw, dev, reps: int) -> dict:

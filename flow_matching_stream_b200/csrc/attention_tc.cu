@@ -14,10 +14,10 @@
 //   * warp 1: MMA issuer. S_i = Q K_iᵀ into one of two TMEM score buffers; P_i (bf16, written
 //     back over its own scores) is the TMEM A operand of O += P_i V_i, V being the MN-major B
 //     operand in shared memory.
-//   * warps 2..5: softmax, one thread per tile row (TMEM lane): one TMEM read of the 64 scores,
-//     row max, exp2 into bf16 P in TMEM, then (after P_{i-1} V_{i-1} has landed) lazy
-//     rescaling of O, only when the running max grows by more than 2^8; final 1/l and
-//     sigmoid(gate) epilogue.
+//   * warps 2..9: softmax, two threads per tile row (TMEM lane), each on 32 of the 64 scores:
+//     half-row max exchanged in shared memory, exp2 into bf16 P in TMEM, then (after
+//     P_{i-1} V_{i-1} has landed) lazy rescaling of its half of O, only when the running max
+//     grows by more than 2^8; final 1/l and sigmoid(gate) epilogue.
 //   * 96 KB of shared memory and 256 TMEM columns per CTA let two CTAs share an SM, so each
 //     SM sub-partition interleaves two independent softmax warps with the MMAs.
 //   * Key tiles whose keys are all padded text are skipped entirely; partially padded tiles and
@@ -39,7 +39,7 @@ namespace {
 constexpr int AD = 128;          // head dim
 constexpr int KT = 64;           // keys per tile
 constexpr int KV_STAGES = 2;
-constexpr int ATT_THREADS = 192;
+constexpr int ATT_THREADS = 320;  // producer, MMA, 8 softmax warps
 constexpr int Q_CHUNK = 128 * 128;                // 128 rows x 64 bf16 (128 B) = 16 KB
 constexpr int Q_BYTES = 2 * Q_CHUNK;              // 32 KB
 constexpr int KV_CHUNK = KT * 128;                // 64 rows x 128 B = 8 KB
@@ -95,12 +95,13 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// exp2 of (v * sl2 - m) for 64 scores, packed to bf16 pairs; returns the row sum of the fp32 values.
+// exp2 of (v * sl2 - m) for NE scores, packed to bf16 pairs; returns the sum of the fp32 values.
+template <int NE>
 __device__ __forceinline__ float exp_tile(const float* v, float sl2, float m, uint32_t* pk) {
   const unsigned long long s2 = f2u(sl2, sl2), nm2 = f2u(-m, -m);
   unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
+  for (int e = 0; e < NE / 2; ++e) {
     float x0, x1;
     u2f(ffma2(f2u(v[2 * e], v[2 * e + 1]), s2, nm2), x0, x1);
     const float a = ex2(x0), c = ex2(x1);
@@ -139,6 +140,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   __shared__ int n_tiles;
   __shared__ int cta_kmin;  // PREFIX: smallest key_end of this CTA's queries (keys below it need no row mask)
   __shared__ uint16_t tiles[MAX_TILES];
+  __shared__ __align__(8) uint64_t ex_bar[4];   // per lane quarter: both halves posted their row max
+  __shared__ __align__(8) uint64_t fin_bar[4];  // per lane quarter: both halves posted their row sum
+  __shared__ float red_max[2][2][128];  // [tile parity][score half][row]: the two halves' row maxima
+  __shared__ float red_l[2][128];       // [score half][row]: partial row sums at the end
 
   constexpr int QPOS = 128 / G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,9 +203,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(&p_full, 128);
+    mbar_init(&p_full, 256);
     mbar_init(&pv_done, 1);
     mbar_init(&drain_bar, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&ex_bar[q], 64);
+      mbar_init(&fin_bar[q], 64);
+    }
     abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
@@ -302,61 +311,68 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       }
     }
   } else {
-    // ---- softmax warps: tile row r = 32 * quarter + lane holds head j*G + r / QPOS at position
-    // p0 + r % QPOS
+    // ---- softmax warps 2..9: tile row r = 32 * quarter + lane holds head j*G + r / QPOS at
+    // position p0 + r % QPOS. Warps w and w+4 share a TMEM lane quarter (the same rows) and split
+    // each row's 64 scores: half 0 takes keys [0, 32) of the tile, half 1 keys [32, 64). They
+    // exchange the row max through shared memory; each keeps its own partial row sum and its
+    // half of the output columns.
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     int row_kend = p.S;
     if constexpr (PREFIX) {
-      const int r = quarter * 32 + lane;
       const int q = p0 + r % QPOS;
       row_kend = q < p.S ? min(max(p.key_end[q], q + 1), p.S) : p.S;
     }
+    constexpr int HK = KT / 2;  // scores per thread and tile
     for (int i = 0; i < n && ok; ++i) {
       const int sb = i & 1;
       if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const int t0 = tiles[i] * KT;
+      const int k0 = t0 + half * HK;  // first key of this thread's half
       const uint32_t sbase = tmem + lane_off + sb * KT;
-      float v[KT];
-      tmem_ld64(sbase, v);
+      float v[HK];
+      tmem_ld32(sbase + half * HK, v);
       if ((t0 < p.T && p.text_mask) || (t0 + KT > p.S)) {  // warp-uniform: only partial tiles mask
-        const uint32_t vm0 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + lane));
-        const uint32_t vm1 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + 32 + lane));
+        const uint32_t vm = __ballot_sync(0xffffffffu, key_valid(p, b, k0 + lane));
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (!((vm0 >> e) & 1u)) v[e] = -INFINITY;
-          if (!((vm1 >> e) & 1u)) v[32 + e] = -INFINITY;
-        }
+        for (int e = 0; e < HK; ++e)
+          if (!((vm >> e) & 1u)) v[e] = -INFINITY;
       }
       if constexpr (PREFIX) {
         if (t0 + KT > cta_kmin) {  // warp-uniform; each row then cuts at its own key_end
-          const int lim = row_kend - t0;
+          const int lim = row_kend - k0;
 #pragma unroll
-          for (int e = 0; e < KT; ++e)
+          for (int e = 0; e < HK; ++e)
             if (e >= lim) v[e] = -INFINITY;
         }
       }
-      // row max: chain k takes v[k], v[k+4], ..., v[k+60] with three-input maxes
-      static_assert(KT == 64, "the max chains below cover 64 scores");
+      // half-row max: chain k takes v[k], v[k+4], ..., v[k+28] with three-input maxes
+      static_assert(HK == 32, "the max chains below cover 32 scores");
       float m4[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         float a = v[k];
 #pragma unroll
-        for (int i = 1; i < 15; i += 2) a = fmax3(a, v[k + 4 * i], v[k + 4 * i + 4]);
-        m4[k] = fmaxf(a, v[k + 60]);
+        for (int t = 1; t < 7; t += 2) a = fmax3(a, v[k + 4 * t], v[k + 4 * t + 4]);
+        m4[k] = fmaxf(a, v[k + 28]);
       }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      // exps against the running max; they only wait for the max when a row's max grows by
-      // more than 2^8 (lazy rescaling), which the warp then handles together
-      uint32_t pk[KT / 2];
-      // while a row has seen no valid key (m = -inf) its exps are taken against 0, so fully
-      // masked scores give 0 rather than NaN
-      float rs = exp_tile(v, sl2, m == -INFINITY ? 0.f : m, pk);
+      red_max[i & 1][half][r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // the arrive also publishes that this half has read its scores: half 1 writes its P over
+      // score columns 16..31, which hold half 0's keys 16..31
+      tc_fence_before();
+      mbar_arrive(&ex_bar[quarter]);
+      // exps against the running max while the partner warp finishes its half
+      uint32_t pk[HK / 2];
+      float rs = exp_tile<HK>(v, sl2, m == -INFINITY ? 0.f : m, pk);
+      if (!mbar_wait(&ex_bar[quarter], i & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      const float mx = fmaxf(red_max[i & 1][0][r], red_max[i & 1][1][r]);
       const float mnew = fmaxf(m, mx * sl2);
       const bool grow = mnew > m + 8.0f;  // m = -inf on the first tile
       float alpha = 1.f;
@@ -366,22 +382,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           alpha = ex2(m - mnew);  // 0 on the first tile
           m = mnew;
         }
-        rs = exp_tile(v, sl2, m == -INFINITY ? 0.f : m, pk);
+        rs = exp_tile<HK>(v, sl2, m == -INFINITY ? 0.f : m, pk);
       }
       l = l * alpha + rs;
-      tmem_st32(sbase, reinterpret_cast<const float*>(pk));  // P_i over the first 32 score columns
+      tmem_st16(sbase + half * (HK / 2), pk);  // P_i (bf16 pairs) over the tile's first 32 columns
       if (i >= 1) {
         // O must hold P_{i-1} V_{i-1} before it is rescaled (also keeps the phase count exact)
         if (!mbar_wait(&pv_done, (i - 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         if (any_grow) {
 #pragma unroll 1
-          for (int c = 0; c < AD / 32; ++c) {
+          for (int c = 0; c < AD / 64; ++c) {
             float o[32];
-            tmem_ld32(tmem + lane_off + O_COL + c * 32, o);
+            const uint32_t oa = tmem + lane_off + O_COL + half * (AD / 2) + c * 32;
+            tmem_ld32(oa, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tmem + lane_off + O_COL + c * 32, o);
+            tmem_st32(oa, o);
           }
         }
       }
@@ -389,31 +406,38 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       tc_fence_before();
       mbar_arrive(&p_full);
     }
+    const int pos = p0 + r % QPOS;
+    const int h = j * G + r / QPOS;
     if (ok && n == 0) {
       // a batch row without any valid key (possible only without image tokens): zeros
-      const int r = quarter * 32 + lane;
-      const int pos = p0 + r % QPOS;
-      const int h = j * G + r / QPOS;
       if (pos < p.S) {
-        uint4* op = reinterpret_cast<uint4*>(p.out + ((long)b * p.S + pos) * p.HD + h * AD);
+        uint4* op = reinterpret_cast<uint4*>(p.out + ((long)b * p.S + pos) * p.HD + h * AD + half * (AD / 2));
 #pragma unroll
-        for (int q = 0; q < AD / 8; ++q) op[q] = make_uint4(0u, 0u, 0u, 0u);
+        for (int q = 0; q < AD / 16; ++q) op[q] = make_uint4(0u, 0u, 0u, 0u);
       }
-    } else if (ok && mbar_wait(&pv_done, (n - 1) & 1, abort)) {
-      tc_fence_after();
-      const int r = quarter * 32 + lane;
-      const int pos = p0 + r % QPOS;
-      const int h = j * G + r / QPOS;
+    } else if (ok) {
+      // the output needs the last P V in O and both halves' row sums
+      ok = mbar_wait(&pv_done, (n - 1) & 1, abort);
+      if (ok) {
+        tc_fence_after();
+        red_l[half][r] = l;
+        mbar_arrive(&fin_bar[quarter]);
+        ok = mbar_wait(&fin_bar[quarter], 0, abort);
+      }
+    }
+    if (ok && n > 0) {
+      const float lt = red_l[0][r] + red_l[1][r];
       const bool row_ok = pos < p.S;
       const long grow_idx = (long)b * p.S + pos;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no readable key: zeros
+      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;  // a row with no readable key: zeros
 #pragma unroll 1
-      for (int c = 0; c < AD / 32; ++c) {
+      for (int c = 0; c < AD / 64; ++c) {
+        const int col = half * (AD / 2) + c * 32;
         float o[32];
-        tmem_ld32(tmem + lane_off + O_COL + c * 32, o);
+        tmem_ld32(tmem + lane_off + O_COL + col, o);
         if (row_ok) {
-          const uint4* gp = reinterpret_cast<const uint4*>(p.gate + grow_idx * p.g_stride + h * AD + c * 32);
-          uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD + c * 32);
+          const uint4* gp = reinterpret_cast<const uint4*>(p.gate + grow_idx * p.g_stride + h * AD + col);
+          uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD + col);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const uint4 gv = __ldg(gp + q);

@@ -99,7 +99,7 @@ def test_attention_bf16_padded_keys_are_ignored(K2):
     np.testing.assert_array_equal(host(out2).reshape(B, S, d.HD), out)
 
 
-@pytest.mark.parametrize("grid", [32, 64])
+@pytest.mark.parametrize("grid", [32, 64, 128])
 def test_attention_sweep_sampled_rows(K2, grid):
     # the attention-only sweep shapes (512 text tokens, random valid length), rows sampled
     wl = KI.attn_sweep(grid)

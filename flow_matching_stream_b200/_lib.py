@@ -55,6 +55,7 @@ SIGNATURES = {
     "krea2_last_error_string": (c_char_p, []),
     "krea2_check_device_error": (c_int, [V]),
     "krea2_workspace_size": (c_size_t, [_PD, c_int, c_int, c_int, c_int]),
+    "krea2_selftest_wait_timeout": (c_int, [c_int, V, V]),
     "krea2_attention_workspace_size": (c_size_t, [_PD, c_int, c_int, c_int, c_int]),
     "krea2_rope_tables": (c_int, [_PD, V, c_int, V, V, V]),
     "krea2_gqa_attention": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V, c_size_t, V]),

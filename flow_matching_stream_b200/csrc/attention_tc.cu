@@ -506,6 +506,30 @@ __global__ void __launch_bounds__(256) qk_prep_kernel(const __nv_bfloat16* __res
 
 KREA2_DEFINE_ERROR_READER(take_device_error_attention)
 
+namespace {
+// One thread waits, with the given limit, on an mbarrier that nothing arrives on: the bounded
+// wait must expire, record the timeout in the device error word and let the kernel return.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, int* waited) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    const bool ok = mbar_wait(&bar, 0, &abort_flag, limit_ns);
+    *waited = ok ? 0 : 1;
+  }
+}
+}  // namespace
+
+int launch_wait_timeout_selftest(unsigned long long limit_ns, int* waited, cudaStream_t stream) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns, waited);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "self-test launch failed: %s", cudaGetErrorString(e));
+  return KREA2_OK;
+}
+
 bool attention_tc_supported(int D, int H, int Hkv) {
   if (D != AD || Hkv <= 0 || H % Hkv) return false;
   const int g = H / Hkv;

@@ -263,6 +263,11 @@ int krea2_check_device_error(void* stream) {
   return KREA2_OK;
 }
 
+int krea2_selftest_wait_timeout(int limit_ms, int* waited, void* stream) {
+  if (limit_ms < 1 || limit_ms > 5000 || !waited) return set_error(KREA2_ERR_ARG, "limit_ms must be 1..5000, waited non-NULL");
+  return launch_wait_timeout_selftest((unsigned long long)limit_ms * 1000000ull, waited, as_stream(stream));
+}
+
 size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype) {
   if (check_dims(dims, dtype) || check_shape(B, T, N)) return 0;
   return ws_layout(dims, B, T, N, dtype).total;

@@ -105,6 +105,7 @@ struct AttnTcArgs {
   const int* key_end;                  // optional (S): query q reads keys [0, key_end[q]) (block-causal)
 };
 bool attention_tc_supported(int D, int H, int Hkv);
+int launch_wait_timeout_selftest(unsigned long long limit_ns, int* waited, cudaStream_t stream);
 int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream);
 // raw [q | k] -> normalised + rotated [q | k] (bf16, row stride (H+Hkv)*128)
 int launch_qk_prep(const void* qkvg, long long stride, int B, int S, int H, int Hkv, float eps, const float* qw,

@@ -122,6 +122,12 @@ const char* krea2_last_error_string(void);
  * entry point that synchronises. */
 int krea2_check_device_error(void* stream);
 
+/* Self-test of the failure detection: launches one kernel that waits, with a limit of limit_ms
+ * (1..5000), on a barrier that nothing arrives on. The bounded wait expires, the kernel writes 1
+ * to *waited (device int) and returns; a following krea2_check_device_error then reports
+ * KREA2_ERR_TIMEOUT and clears the error word. The context stays usable. */
+int krea2_selftest_wait_timeout(int limit_ms, int* waited, void* stream);
+
 /* Bytes of device workspace that krea2_block_forward / krea2_backbone_forward need for
  * these shapes (0 on invalid arguments). The workspace must be 256-byte aligned. */
 size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype);

@@ -86,25 +86,61 @@ def peaks() -> dict:
         return dict(FALLBACK, source="fallback")
 
 
-def kernel_source_hash() -> str:
+# Source files that fix each block step's kernel and its launch shape. A recorded DRAM figure
+# is only valid while these files are unchanged.
+_GEMM_SOURCES = ("gemm_tcgen05.cu", "krea2_device.cuh", "krea2_internal.h")
+KERNEL_SOURCES = {
+    "qkv_proj": _GEMM_SOURCES, "out_proj_resid": _GEMM_SOURCES, "gate_up_swiglu": _GEMM_SOURCES,
+    "down_proj_resid": _GEMM_SOURCES,
+    "attention": ("attention_tc.cu", "krea2_device.cuh", "krea2_internal.h"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "flow_matching_stream_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(KERNEL_SOURCES[kernel]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernels."""
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f).get("kernels", {}).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not rec or kernel not in KERNEL_SOURCES or rec.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def record_traffic(entries) -> None:
+    """Store ncu DRAM bytes per launch (read + write) for block steps, stamped with their source hash.
+
+    entries: "kernel=bytes[:profile]" strings, profile naming the summary under profiles/."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
-        return None
-    if t.get("source_hash") != kernel_source_hash():
-        return None
-    return t.get("kernels", {}).get(kernel, {}).get("dram_bytes_per_launch")
+        t = {}
+    t["_source"] = ("dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu captures at the "
+                    "backbone block shape; an entry is valid only while its kernel sources hash to source_hash")
+    kernels = t.setdefault("kernels", {})
+    for e in entries:
+        name, rest = e.split("=", 1)
+        nbytes, _, profile = rest.partition(":")
+        if name not in KERNEL_SOURCES:
+            raise SystemExit(f"unknown block step {name!r}; one of {sorted(KERNEL_SOURCES)}")
+        kernels[name] = {"dram_bytes_per_launch": int(nbytes), "source_hash": kernel_source_hash(name)}
+        if profile:
+            kernels[name]["profile"] = profile
+    t.pop("source_hash", None)
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(t, f, indent=1, sort_keys=True)
+        f.write("\n")
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -662,9 +698,14 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("native", "reference"), default="native")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--record-traffic", nargs="+", metavar="STEP=BYTES[:PROFILE]", default=None,
+                    help="store ncu DRAM bytes per launch for block steps and exit")
     ap.add_argument("--kernel-case", choices=KERNEL_CASES, default=None,
                     help="run one kernel at the backbone block shape (for profiler captures)")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic)
+        return
     if args.kernel_case:
         run_kernel_case(args.kernel_case, args.steps)
         return

@@ -30,8 +30,9 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 // Row tiles per raster group: as many as keep the group's A tiles (128 x K bf16 each) within
-// about 48 MB of L2, so W streams from HBM about once per group pass.
-constexpr size_t GROUP_A_BYTES = 48ull << 20;
+// about 24 MB of L2, so W streams from HBM once per group pass. Larger groups measured more
+// DRAM re-reads of W, not fewer: their A tiles did not stay resident.
+constexpr size_t GROUP_A_BYTES = 24ull << 20;
 constexpr int GEMM_THREADS = 192;
 
 template <int BN>

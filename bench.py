@@ -358,6 +358,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     sampler = time_sampler(K2, torch, d, mw, dev)
     text = time_text_fusion(K2, torch, dev, args.steps)
     sweep = time_attention_sweep(K2, torch, dev, args.steps, pk)
+    kv_step = time_kv_cache_step(K2, torch, dev, args.steps, pk)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -373,6 +374,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         "sampler_1024sq": sampler,
         "text_fusion_once_per_prompt": text,
         "attention_sweep": sweep,
+        "kv_cache_step_attention": kv_step,
         "pct_of_tensor_peak": {"burst": value / world / pk["bf16_tflops"],
                                "sustained": value / world / pk["bf16_tflops_sustained"]},
         "block_1024sq_cfg": cfg_res,
@@ -524,6 +526,55 @@ def time_attention_sweep(K2, torch, dev, steps: int, pk: dict) -> list:
     return out
 
 
+def time_kv_cache_step(K2, torch, dev, steps: int, pk: dict) -> dict:
+    """One denoising step's attention of the block-causal variant with a key/value cache: the
+    prompt (512 text tokens, random valid length) and a 64x64 condition image are cached once;
+    each step appends the 64x64 target image's keys and values and runs its 4096 queries over all
+    8704 keys (krea2_kv_cache_append + krea2_gqa_attention_kv_cache). FLOPs count valid keys only."""
+    wl = KI.backbone_1024()
+    d = wl.dims
+    T, Ni = wl.T, wl.N
+    P, Nq = T + Ni, Ni
+    L = P + Nq
+    g = torch.Generator(device=dev).manual_seed(31)
+    x = torch.randn(L, d.qkvg_cols, device=dev, generator=g).to(torch.bfloat16)
+    qw = torch.randn(d.D, device=dev, generator=g) * 0.1
+    kw = torch.randn(d.D, device=dev, generator=g) * 0.1
+    pos = np.concatenate([KI.position_ids(T, 64, 64), KI.position_ids(0, 64, 64)]).astype(np.float32)
+    pos[P:, 0] = 1.0  # the target image sits one step along the first axis
+    cs = torch.empty(L, d.D // 2, device=dev)
+    sn = torch.empty_like(cs)
+    K2.rope_tables(d, torch.from_numpy(pos).to(dev), cs, sn)
+    mask = torch.from_numpy(wl.mask().astype(np.uint8)).to(dev)
+    kc = torch.empty(1, L, d.KVD, device=dev, dtype=torch.bfloat16)
+    vc = torch.empty_like(kc)
+    x_prefix, x_new = x[:P].contiguous(), x[P:].contiguous()
+    K2.kv_cache_append(d, 1, P, 0, x_prefix, kw, cs[:P], sn[:P], kc, vc)
+    o = torch.empty(Nq, d.HD, device=dev, dtype=torch.bfloat16)
+    ws = torch.empty(K2.kv_cache_attention_workspace_size(d, 1, Nq, torch.bfloat16), dtype=torch.uint8, device=dev)
+    cs_new, sn_new = cs[P:].contiguous(), sn[P:].contiguous()
+
+    def run():
+        K2.kv_cache_append(d, 1, Nq, P, x_new, kw, cs_new, sn_new, kc, vc)
+        K2.gqa_attention_kv_cache(d, 1, T, L, Nq, x_new, qw, cs_new, sn_new, mask, kc, vc, None, o, ws)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    K2.check_device_error()
+    ms = e0.elapsed_time(e1) / steps
+    fl = 4.0 * d.D * d.H * Nq * (wl.lengths[0] + Ni + Nq)
+    return {"workload": "block-causal step with cached prompt + 64x64 condition image, 64x64 target",
+            "new_tokens": Nq, "keys": L, "valid_text": int(wl.lengths[0]), "ms": ms,
+            "tflops": fl / (ms / 1e3) / 1e12, "frac_burst": fl / (ms / 1e3) / 1e12 / pk["bf16_tflops"]}
+
+
 def traced_block_kernels(K2, torch, d, B, T, N, lengths, bw, dev, reps: int) -> dict:
     S = T + N
     pk = peaks()
@@ -620,7 +671,7 @@ def run_reference(args, rank: int) -> None:
 
 # ----------------------------------------------------------------------------- single-kernel cases
 
-KERNEL_CASES = ("gate_up", "qkv", "down", "attention", "norm")
+KERNEL_CASES = ("gate_up", "qkv", "out_proj", "down", "attention", "norm")
 
 
 def run_kernel_case(name: str, steps: int) -> None:
@@ -640,14 +691,15 @@ def run_kernel_case(name: str, steps: int) -> None:
     def rnd(*shape, scale=1.0):
         return (torch.randn(*shape, device=dev, generator=g) * scale).to(bf)
 
-    if name in ("gate_up", "qkv", "down"):
+    if name in ("gate_up", "qkv", "out_proj", "down"):
         K = d.F if name == "down" else d.C
-        Nw = {"gate_up": 2 * d.F, "qkv": d.qkvg_cols, "down": d.C}[name]
+        Nw = {"gate_up": 2 * d.F, "qkv": d.qkvg_cols, "out_proj": d.C, "down": d.C}[name]
         A, W = rnd(M, K), rnd(Nw, K, scale=K ** -0.5)
-        if name == "down":
+        if name in ("out_proj", "down"):
             out = torch.zeros(M, Nw, device=dev)
             gate = torch.randn(B, 6 * d.C, device=dev)
-            fn = lambda: K2.linear(K2.KREA2_EPI_RESID, A, W, out, gate=gate.view(-1)[5 * d.C:], rows_per_batch=S,
+            g_off = (5 if name == "down" else 2) * d.C  # gate_mlp / gate_msa of the modulation
+            fn = lambda: K2.linear(K2.KREA2_EPI_RESID, A, W, out, gate=gate.view(-1)[g_off:], rows_per_batch=S,
                                    gate_stride=6 * d.C)
         elif name == "gate_up":
             out = torch.empty(M, d.F, device=dev, dtype=bf)

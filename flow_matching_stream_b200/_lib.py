@@ -76,6 +76,10 @@ SIGNATURES = {
     "krea2_text_fusion_workspace_size": (c_size_t, [_PTD, c_int, c_int, c_int]),
     "krea2_text_fusion": (c_int, [_PTD, c_int, c_int, c_int, V, V, _PTW, V, V, c_size_t, V]),
     "krea2_block_causal_key_end": (c_int, [V, c_int, V]),
+    "krea2_kv_cache_append": (c_int, [_PD, c_int, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V]),
+    "krea2_kv_cache_attention_workspace_size": (c_size_t, [_PD, c_int, c_int, c_int]),
+    "krea2_gqa_attention_kv_cache": (c_int, [_PD, c_int, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, c_int, V,
+                                             V, V, c_size_t, V]),
     "krea2_gqa_attention_block_causal": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V, V,
                                                  c_size_t, V]),
     "krea2_gqa_attention_noalloc": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V]),

@@ -32,7 +32,7 @@
 namespace krea2 {
 
 int make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t batches,
-                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows);
+                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows, uint64_t batch_rows);
 
 namespace {
 
@@ -56,12 +56,14 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AD, 0, 1);
 
 struct AttnCore {
   int B, T, N, S, Hkv, HD;
+  int Sq;     // query rows per batch row (S, or the new tokens of a key/value cache step)
+  int q_off;  // key position of query row 0 (0, or L - Sq for a cache step)
   const uint8_t* text_mask;
   const __nv_bfloat16* gate;  // gate column block base (row stride g_stride)
   long long g_stride;
   __nv_bfloat16* out;         // (B*S, HD)
   float scale_log2;
-  const int* key_end;         // PREFIX: query q reads keys [0, key_end[q]) only (same for all batch rows)
+  const int* key_end;         // PREFIX: query row q reads keys [0, key_end[q]) only (same for all batch rows)
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -159,8 +161,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       int hi = 0, lo = p.S;
       for (int i = lane; i < QPOS; i += 32) {
         const int q = p0 + i;
-        if (q < p.S) {
-          const int e = min(max(p.key_end[q], q + 1), p.S);
+        if (q < p.Sq) {
+          const int e = min(max(p.key_end[q], p.q_off + q + 1), p.S);
           hi = max(hi, e);
           lo = min(lo, e);
         }
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     int row_kend = p.S;
     if constexpr (PREFIX) {
       const int q = p0 + r % QPOS;
-      row_kend = q < p.S ? min(max(p.key_end[q], q + 1), p.S) : p.S;
+      row_kend = q < p.Sq ? min(max(p.key_end[q], p.q_off + q + 1), p.S) : p.S;
     }
     constexpr int HK = KT / 2;  // scores per thread and tile
     for (int i = 0; i < n && ok; ++i) {
@@ -410,8 +412,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     const int h = j * G + r / QPOS;
     if (ok && n == 0) {
       // a batch row without any valid key (possible only without image tokens): zeros
-      if (pos < p.S) {
-        uint4* op = reinterpret_cast<uint4*>(p.out + ((long)b * p.S + pos) * p.HD + h * AD + half * (AD / 2));
+      if (pos < p.Sq) {
+        uint4* op = reinterpret_cast<uint4*>(p.out + ((long)b * p.Sq + pos) * p.HD + h * AD + half * (AD / 2));
 #pragma unroll
         for (int q = 0; q < AD / 16; ++q) op[q] = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -427,8 +429,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     }
     if (ok && n > 0) {
       const float lt = red_l[0][r] + red_l[1][r];
-      const bool row_ok = pos < p.S;
-      const long grow_idx = (long)b * p.S + pos;
+      const bool row_ok = pos < p.Sq;
+      const long grow_idx = (long)b * p.Sq + pos;
       const float inv_l = lt > 0.f ? 1.f / lt : 0.f;  // a row with no readable key: zeros
 #pragma unroll 1
       for (int c = 0; c < AD / 64; ++c) {
@@ -469,8 +471,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   }
 }
 
+// One warp normalises one 128-wide head (RMSNorm over head_dim with weight (1 + w), page §四.3)
+// and rotates it by the position's RoPE angles (adjacent pairs); each lane holds 4 columns.
+__device__ __forceinline__ uint2 norm_rope_head(const __nv_bfloat16* x, const float* w, const float* cs,
+                                               const float* sn, int pos, float eps, int lane) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(x + lane * 4);
+  float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+  const float ss = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
+  const float r = rsqrtf(ss / (float)AD + eps);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] *= r * (1.f + w[lane * 4 + e]);
+  const float c0 = cs[(long)pos * (AD / 2) + lane * 2], s0 = sn[(long)pos * (AD / 2) + lane * 2];
+  const float c1 = cs[(long)pos * (AD / 2) + lane * 2 + 1], s1 = sn[(long)pos * (AD / 2) + lane * 2 + 1];
+  uint2 o;
+  o.x = pack_bf16x2(v[0] * c0 - v[1] * s0, v[1] * c0 + v[0] * s0);
+  o.y = pack_bf16x2(v[2] * c1 - v[3] * s1, v[3] * c1 + v[2] * s1);
+  return o;
+}
+
 // Raw projection -> RMS-normalised, rotated q and k (bf16), one warp per (row, head).
-// dst row layout: [q heads (H*D) | k heads (Hkv*D)].
+// dst row layout: [q heads (H*D) | k heads (Hkv*D)]; Hkv = 0 prepares q only.
 __global__ void __launch_bounds__(256) qk_prep_kernel(const __nv_bfloat16* __restrict__ src, long long src_stride,
                                                       int S, int H, int Hkv, float eps,
                                                       const float* __restrict__ qw, const float* __restrict__ kw,
@@ -483,23 +503,32 @@ __global__ void __launch_bounds__(256) qk_prep_kernel(const __nv_bfloat16* __res
   const long row = gw / heads;
   const int hh = (int)(gw % heads);
   const int pos = (int)(row % S);
-  const bool is_q = hh < H;
-  const float* w = is_q ? qw : kw;
-  const __nv_bfloat16* x = src + row * src_stride + (long)hh * AD + lane * 4;
-  const uint2 raw = *reinterpret_cast<const uint2*>(x);
-  float v[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
-  const float ss = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
-  const float r = rsqrtf(ss / (float)AD + eps);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) v[e] *= r * (1.f + w[lane * 4 + e]);
-  const float c0 = cs[(long)pos * (AD / 2) + lane * 2], s0 = sn[(long)pos * (AD / 2) + lane * 2];
-  const float c1 = cs[(long)pos * (AD / 2) + lane * 2 + 1], s1 = sn[(long)pos * (AD / 2) + lane * 2 + 1];
-  const float y0 = v[0] * c0 - v[1] * s0, y1 = v[1] * c0 + v[0] * s0;
-  const float y2 = v[2] * c1 - v[3] * s1, y3 = v[3] * c1 + v[2] * s1;
-  uint2 o;
-  o.x = pack_bf16x2(y0, y1);
-  o.y = pack_bf16x2(y2, y3);
+  const uint2 o = norm_rope_head(src + row * src_stride + (long)hh * AD, hh < H ? qw : kw, cs, sn, pos, eps, lane);
   *reinterpret_cast<uint2*>(dst + row * (long)(heads * AD) + (long)hh * AD + lane * 4) = o;
+}
+
+// Keys and values of n new tokens into a key/value cache, one warp per (token, KV head): k is
+// normalised and rotated like the attention's keys, v is copied as projected. Token i of batch
+// row b lands in cache row b * capacity + row0 + i.
+__global__ void __launch_bounds__(256) kv_append_kernel(const __nv_bfloat16* __restrict__ src, long long src_stride,
+                                                        int n, int H, int Hkv, float eps,
+                                                        const float* __restrict__ kw, const float* __restrict__ cs,
+                                                        const float* __restrict__ sn, long rows,
+                                                        __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc,
+                                                        int row0, int capacity) {
+  const long gw = (long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows * Hkv) return;
+  const long row = gw / Hkv;
+  const int hh = (int)(gw % Hkv);
+  const int i = (int)(row % n);
+  const long drow = (row / n) * capacity + row0 + i;
+  const __nv_bfloat16* x = src + row * src_stride;
+  const uint2 ko = norm_rope_head(x + (long)(H + hh) * AD, kw, cs, sn, i, eps, lane);
+  const uint2 vo = *reinterpret_cast<const uint2*>(x + (long)(H + Hkv + hh) * AD + lane * 4);
+  const long d = drow * (long)(Hkv * AD) + (long)hh * AD + lane * 4;
+  *reinterpret_cast<uint2*>(kc + d) = ko;
+  *reinterpret_cast<uint2*>(vc + d) = vo;
 }
 
 }  // namespace
@@ -550,21 +579,26 @@ int launch_attention_g(const AttnTcArgs& a, cudaStream_t stream) {
     attr_done = true;
   }
   const int S = a.T + a.N;
+  const int Sq = a.Sq > 0 ? a.Sq : S;
+  const long long kv_rows = a.kv_batch_rows > 0 ? a.kv_batch_rows : S;
   if ((S + KT - 1) / KT > MAX_TILES) return set_error(KREA2_ERR_UNSUPPORTED, "sequence longer than %d", MAX_TILES * KT);
+  if (Sq > S || a.q_off < 0 || a.q_off + Sq > S)
+    return set_error(KREA2_ERR_ARG, "query rows [%d, %d) lie outside the %d keys", a.q_off, a.q_off + Sq, S);
   CUtensorMap tq, tk, tv;
   int rc;
-  if ((rc = make_tmap_bf16_3d(&tq, a.q, (uint64_t)a.H * AD, S, a.B, a.q_stride, 64, QPOS))) return rc;
-  if ((rc = make_tmap_bf16_3d(&tk, a.k, (uint64_t)a.Hkv * AD, S, a.B, a.k_stride, 64, KT))) return rc;
-  if ((rc = make_tmap_bf16_3d(&tv, a.v, (uint64_t)a.Hkv * AD, S, a.B, a.v_stride, 64, KT))) return rc;
+  if ((rc = make_tmap_bf16_3d(&tq, a.q, (uint64_t)a.H * AD, Sq, a.B, a.q_stride, 64, QPOS, Sq))) return rc;
+  if ((rc = make_tmap_bf16_3d(&tk, a.k, (uint64_t)a.Hkv * AD, S, a.B, a.k_stride, 64, KT, kv_rows))) return rc;
+  if ((rc = make_tmap_bf16_3d(&tv, a.v, (uint64_t)a.Hkv * AD, S, a.B, a.v_stride, 64, KT, kv_rows))) return rc;
   AttnCore p{};
   p.B = a.B; p.T = a.T; p.N = a.N; p.S = S; p.Hkv = a.Hkv; p.HD = a.H * AD;
+  p.Sq = Sq; p.q_off = a.q_off;
   p.text_mask = a.text_mask;
   p.gate = reinterpret_cast<const __nv_bfloat16*>(a.g);
   p.g_stride = a.g_stride;
   p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)AD);
   p.key_end = a.key_end;
-  dim3 grid((S + QPOS - 1) / QPOS, a.Hkv, a.B);
+  dim3 grid((Sq + QPOS - 1) / QPOS, a.Hkv, a.B);
   attn_gqa_tc_kernel<G, PREFIX><<<grid, ATT_THREADS, ATT_SMEM, stream>>>(tq, tk, tv, p);
   count_launch();
   cudaError_t e = cudaGetLastError();
@@ -587,6 +621,20 @@ int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
     case 2: return launch_attention_g<2, false>(a, stream);
     default: return launch_attention_g<4, false>(a, stream);
   }
+}
+
+int launch_kv_append(const void* qkvg, long long stride, int B, int n, int H, int Hkv, float eps, const float* kw,
+                     const float* cs, const float* sn, void* k_cache, void* v_cache, int row0, int capacity,
+                     cudaStream_t stream) {
+  const long rows = (long)B * n;
+  const long warps = rows * Hkv;
+  kv_append_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(qkvg), stride, n, H, Hkv, eps, kw, cs, sn, rows,
+      reinterpret_cast<__nv_bfloat16*>(k_cache), reinterpret_cast<__nv_bfloat16*>(v_cache), row0, capacity);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "kv_append launch failed: %s", cudaGetErrorString(e));
+  return KREA2_OK;
 }
 
 int launch_qk_prep(const void* qkvg, long long stride, int B, int S, int H, int Hkv, float eps, const float* qw,

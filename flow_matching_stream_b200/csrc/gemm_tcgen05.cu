@@ -385,14 +385,18 @@ int make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
 // Row-major bf16 matrix viewed as (batches, rows, cols) with `row_stride_elems` between rows and
 // rows*row_stride between batches; box (box_cols x box_rows x 1), 128-byte swizzle. Rows past
 // `rows` in a batch read as zero.
+// (cols, rows, batches) view with batch b starting batch_rows rows after batch b-1 (batch_rows >=
+// rows); rows at or beyond `rows` read as zeros, also when the buffer holds more.
 int make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t rows, uint64_t batches,
-                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows) {
+                      uint64_t row_stride_elems, uint32_t box_cols, uint32_t box_rows, uint64_t batch_rows) {
   auto enc = get_encode_fn();
   if (!enc) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((row_stride_elems * 2) & 15))
     return set_error(KREA2_ERR_ARG, "TMA operand must be 16-byte aligned with a 16-byte multiple row stride");
   cuuint64_t dims[3] = {cols, rows, batches};
-  cuuint64_t strides[2] = {row_stride_elems * 2, row_stride_elems * 2 * rows};
+  if (batch_rows < rows) return set_error(KREA2_ERR_ARG, "batch stride of %llu rows is below the %llu rows read",
+                                          (unsigned long long)batch_rows, (unsigned long long)rows);
+  cuuint64_t strides[2] = {row_stride_elems * 2, row_stride_elems * 2 * batch_rows};
   cuuint32_t box[3] = {box_cols, box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,

@@ -348,6 +348,63 @@ int krea2_gqa_attention_block_causal(const Krea2Dims* dims, int B, int T, int N,
   return attention_raw(ap, dtype, workspace, as_stream(stream), key_end);
 }
 
+size_t krea2_kv_cache_attention_workspace_size(const Krea2Dims* dims, int B, int Nq, int dtype) {
+  if (check_dims(dims, dtype) || B <= 0 || Nq <= 0 || dtype != KREA2_BF16 ||
+      !attention_tc_supported(dims->D, dims->H, dims->Hkv))
+    return 0;
+  return (size_t)B * Nq * (size_t)dims->H * dims->D * 2;
+}
+
+int krea2_kv_cache_append(const Krea2Dims* dims, int B, int n, int row0, int capacity, int dtype, const void* qkvg,
+                          const float* k_norm_w, const float* cos, const float* sin, void* k_cache, void* v_cache,
+                          void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc) return rc;
+  if (B <= 0 || n <= 0 || row0 < 0 || capacity <= 0 || (long long)row0 + n > capacity)
+    return set_error(KREA2_ERR_ARG, "need B >= 1, n >= 1 and 0 <= row0, row0 + n <= capacity (%d + %d > %d)", row0, n,
+                     capacity);
+  if (!qkvg || !k_norm_w || !cos || !sin || !k_cache || !v_cache) return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (dtype != KREA2_BF16 || !attention_tc_supported(dims->D, dims->H, dims->Hkv))
+    return set_error(KREA2_ERR_UNSUPPORTED, "the key/value cache needs bf16, D=128, H/Hkv in {1,2,4}");
+  if ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15)
+    return set_error(KREA2_ERR_ARG, "k_cache and v_cache must be 16-byte aligned");
+  const long long QC = 2LL * dims->H * dims->D + 2LL * dims->Hkv * dims->D;
+  return launch_kv_append(qkvg, QC, B, n, dims->H, dims->Hkv, dims->eps, k_norm_w, cos, sin, k_cache, v_cache, row0,
+                          capacity, as_stream(stream));
+}
+
+int krea2_gqa_attention_kv_cache(const Krea2Dims* dims, int B, int T, int L, int Nq, int dtype, const void* qkvg,
+                                 const float* q_norm_w, const float* cos, const float* sin, const uint8_t* text_mask,
+                                 const void* k_cache, const void* v_cache, int capacity, const int32_t* key_end,
+                                 void* out, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_dims(dims, dtype);
+  if (rc) return rc;
+  if (B <= 0 || T < 0 || Nq <= 0 || L < Nq || T > L || capacity < L)
+    return set_error(KREA2_ERR_ARG, "need B >= 1, 1 <= Nq <= L, 0 <= T <= L and capacity >= L");
+  if (!qkvg || !q_norm_w || !cos || !sin || !k_cache || !v_cache || !out)
+    return set_error(KREA2_ERR_ARG, "NULL pointer");
+  if (dtype != KREA2_BF16 || !attention_tc_supported(dims->D, dims->H, dims->Hkv))
+    return set_error(KREA2_ERR_UNSUPPORTED, "the key/value cache needs bf16, D=128, H/Hkv in {1,2,4}");
+  const size_t need = krea2_kv_cache_attention_workspace_size(dims, B, Nq, dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (ws_bytes < need) return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  const cudaStream_t s = as_stream(stream);
+  const int H = dims->H, Hkv = dims->Hkv, D = dims->D;
+  const long long QC = 2LL * H * D + 2LL * Hkv * D;
+  // q of the new tokens only (Hkv = 0: no k heads in the prepared rows)
+  if ((rc = launch_qk_prep(qkvg, QC, B, Nq, H, 0, dims->eps, q_norm_w, q_norm_w, cos, sin, workspace, s))) return rc;
+  AttnTcArgs a{};
+  a.B = B; a.T = T; a.N = L - T; a.H = H; a.Hkv = Hkv;
+  a.q = workspace; a.q_stride = (long long)H * D;
+  a.k = k_cache; a.k_stride = (long long)Hkv * D;
+  a.v = v_cache; a.v_stride = (long long)Hkv * D;
+  a.g = reinterpret_cast<const __nv_bfloat16*>(qkvg) + (long long)(H + 2 * Hkv) * D; a.g_stride = QC;
+  a.text_mask = T > 0 ? text_mask : nullptr; a.out = out; a.key_end = key_end;
+  a.Sq = Nq; a.q_off = L - Nq; a.kv_batch_rows = capacity;
+  return attention_tc_core(a, s);
+}
+
 int krea2_modulated_rmsnorm(const Krea2Dims* dims, int B, int S, int dtype, const float* h, const float* norm_w,
                             const float* temb, const float* table, int chunk, void* out, void* stream) {
   int rc = check_dims(dims, dtype);

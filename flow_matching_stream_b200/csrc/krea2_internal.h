@@ -102,11 +102,19 @@ struct AttnTcArgs {
   const void* g; long long g_stride;
   const uint8_t* text_mask;
   void* out;                           // (B*S, H*128) bf16
-  const int* key_end;                  // optional (S): query q reads keys [0, key_end[q]) (block-causal)
+  const int* key_end;                  // optional (Sq): query row q reads keys [0, key_end[q]) (block-causal)
+  int Sq;                              // query rows per batch row; 0 means S = T + N
+  int q_off;                           // key position of query row 0 (queries are keys [q_off, q_off + Sq))
+  long long kv_batch_rows;             // rows between batch rows of k and v; 0 means S
 };
 bool attention_tc_supported(int D, int H, int Hkv);
 int launch_wait_timeout_selftest(unsigned long long limit_ns, int* waited, cudaStream_t stream);
 int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream);
+// raw k and v of n tokens -> rows [row0, row0 + n) of every batch row of a key/value cache
+// (k RMS-normalised and rotated, v copied; bf16, (B, capacity, Hkv*128))
+int launch_kv_append(const void* qkvg, long long stride, int B, int n, int H, int Hkv, float eps, const float* kw,
+                     const float* cs, const float* sn, void* k_cache, void* v_cache, int row0, int capacity,
+                     cudaStream_t stream);
 // raw [q | k] -> normalised + rotated [q | k] (bf16, row stride (H+Hkv)*128)
 int launch_qk_prep(const void* qkvg, long long stride, int B, int S, int H, int Hkv, float eps, const float* qw,
                    const float* kw, const float* cs, const float* sn, void* dst, cudaStream_t stream);

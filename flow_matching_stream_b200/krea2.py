@@ -19,7 +19,8 @@ from ._lib import KREA2_BF16, KREA2_F32, KREA2_EPI_RESID, KREA2_EPI_STORE, KREA2
 
 __all__ = [
     "Krea2Error", "lib", "dims_struct", "dtype_code", "workspace_size", "attention_workspace_size",
-    "rope_tables", "gqa_attention", "gqa_attention_noalloc", "block_causal_key_end", "gqa_attention_block_causal", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
+    "rope_tables", "gqa_attention", "gqa_attention_noalloc", "block_causal_key_end", "gqa_attention_block_causal",
+    "kv_cache_append", "kv_cache_attention_workspace_size", "gqa_attention_kv_cache", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
     "text_dims_struct", "TextWeights", "text_fusion_workspace_size", "text_fusion",
     "shift_mu", "sigma_schedule", "euler_cfg_step", "sample_workspace_size", "sample",
     "block_forward", "block_forward_traced", "BLOCK_STEPS", "launch_count", "backbone_forward", "check_device_error", "BlockWeights", "ModelWeights",
@@ -148,6 +149,37 @@ def gqa_attention_block_causal(dims, B: int, T: int, N: int, qkvg: torch.Tensor,
     _check(lib().krea2_gqa_attention_block_causal(
         ctypes.byref(dims_struct(dims)), B, T, N, dtype_code(qkvg.dtype), _p(qkvg), _p(q_norm_w), _p(k_norm_w),
         _p(cos), _p(sin), _p(text_mask), _p(key_end), _p(out), _p(workspace),
+        workspace.numel() * workspace.element_size(), _s(stream)))
+
+
+def kv_cache_append(dims, B: int, n: int, row0: int, qkvg: torch.Tensor, k_norm_w: torch.Tensor, cos: torch.Tensor,
+                    sin: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, stream=None) -> None:
+    """Keys and values of n tokens into rows [row0, row0 + n) of a (B, capacity, Hkv*D) cache."""
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _want(t, qkvg.dtype, name)
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 3 or k_cache.shape[0] != B:
+        raise ValueError("k_cache and v_cache must both be (B, capacity, Hkv*D)")
+    _check(lib().krea2_kv_cache_append(ctypes.byref(dims_struct(dims)), B, n, row0, k_cache.shape[1],
+                                       dtype_code(qkvg.dtype), _p(qkvg), _p(k_norm_w), _p(cos), _p(sin),
+                                       _p(k_cache), _p(v_cache), _s(stream)))
+
+
+def kv_cache_attention_workspace_size(dims, B: int, Nq: int, dtype: torch.dtype) -> int:
+    return int(lib().krea2_kv_cache_attention_workspace_size(ctypes.byref(dims_struct(dims)), B, Nq,
+                                                             dtype_code(dtype)))
+
+
+def gqa_attention_kv_cache(dims, B: int, T: int, L: int, Nq: int, qkvg: torch.Tensor, q_norm_w: torch.Tensor,
+                           cos: torch.Tensor, sin: torch.Tensor, text_mask: Optional[torch.Tensor],
+                           k_cache: torch.Tensor, v_cache: torch.Tensor, key_end: Optional[torch.Tensor],
+                           out: torch.Tensor, workspace: torch.Tensor, stream=None) -> None:
+    """Attention of the Nq tokens at key positions [L - Nq, L) over the first L cached keys."""
+    if key_end is not None:
+        _want(key_end, torch.int32, "key_end")
+    _want(out, qkvg.dtype, "out")
+    _check(lib().krea2_gqa_attention_kv_cache(
+        ctypes.byref(dims_struct(dims)), B, T, L, Nq, dtype_code(qkvg.dtype), _p(qkvg), _p(q_norm_w), _p(cos),
+        _p(sin), _p(text_mask), _p(k_cache), _p(v_cache), k_cache.shape[1], _p(key_end), _p(out), _p(workspace),
         workspace.numel() * workspace.element_size(), _s(stream)))
 
 

@@ -200,6 +200,46 @@ int krea2_gqa_attention_block_causal(const Krea2Dims* dims, int B, int T, int N,
                                      const int32_t* key_end, void* out, void* workspace,
                                      size_t ws_bytes, void* stream);
 
+/* Key/value cache of the block-causal variant (page "QwenImage21Transformer2DModel": with
+ * causal_condition the text and condition-image tokens are modulated from t = 0, so their keys
+ * and values do not change between denoising steps and are kept in a kv_cache). The cache holds,
+ * per batch row, `capacity` rows of keys and of values: k_cache and v_cache are
+ * (B, capacity, Hkv*D) bf16 DEVICE buffers, 16-byte aligned, owned by the caller.
+ *
+ * krea2_kv_cache_append stores the keys and values of n tokens in rows [row0, row0 + n) of every
+ * batch row: k RMS-normalised over head_dim with weight (1 + k_norm_w) and rotated by (cos, sin),
+ * v as projected (the same k and v krea2_gqa_attention computes).
+ *   qkvg (B*n, H*D + 2*Hkv*D + H*D) raw fused projection of the n tokens; only the k and v
+ *   columns are read. cos, sin (n, D/2) fp32: RoPE tables of the n tokens.
+ * Returns KREA2_ERR_ARG unless 0 <= row0 and row0 + n <= capacity; tensor-core shapes only
+ * (bf16, D = 128, H/Hkv in {1, 2, 4}), else KREA2_ERR_UNSUPPORTED. */
+int krea2_kv_cache_append(const Krea2Dims* dims, int B, int n, int row0, int capacity, int dtype,
+                          const void* qkvg, const float* k_norm_w, const float* cos, const float* sin,
+                          void* k_cache, void* v_cache, void* stream);
+
+/* Attention of Nq new tokens over the first L cached keys, on the tensor-core attention kernel.
+ * The new tokens are the keys at positions [L - Nq, L); their keys and values must already be in
+ * the cache (krea2_kv_cache_append with row0 = L - Nq). Keys [0, T) are text tokens, and
+ * text_mask (B, T) uint8 (NULL: all valid) removes padded ones.
+ *   key_end NULL: every new token reads all L keys. That is the last image block of a
+ *     block-causal sequence (the image being denoised), which sees every earlier token and its
+ *     own block.
+ *   key_end (Nq) int32 DEVICE: new token i reads keys [0, key_end[i]) (absolute positions, e.g.
+ *     rows L - Nq .. L - 1 of krea2_block_causal_key_end over the whole sequence); a key_end
+ *     below the token's own position + 1 is raised to it.
+ *   qkvg (B*Nq, H*D + 2*Hkv*D + H*D) raw fused projection of the new tokens: q is RMS-normalised
+ *     (1 + q_norm_w) and rotated by cos, sin (Nq, D/2); the gate columns gate the output.
+ *   out (B*Nq, H*D) bf16: sigmoid(gate) * attention, heads merged. A token with no readable key
+ *     outputs zeros.
+ *   workspace: krea2_kv_cache_attention_workspace_size bytes, 256-byte aligned (prepared q).
+ * Returns KREA2_ERR_ARG unless 1 <= Nq <= L, 0 <= T <= L and capacity >= L. */
+size_t krea2_kv_cache_attention_workspace_size(const Krea2Dims* dims, int B, int Nq, int dtype);
+int krea2_gqa_attention_kv_cache(const Krea2Dims* dims, int B, int T, int L, int Nq, int dtype,
+                                 const void* qkvg, const float* q_norm_w, const float* cos, const float* sin,
+                                 const uint8_t* text_mask, const void* k_cache, const void* v_cache,
+                                 int capacity, const int32_t* key_end, void* out, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
 /* Shared modulation of one block plus its table, then a modulated RMSNorm ([ARCH] §四.2,
  * §四.4): with mod = temb (B, 6C) viewed as (B, 6, C) plus table (6, C),
  *   out[b, s] = (1 + mod[b, chunk]) * rms(h[b, s]) * (1 + norm_w) + mod[b, chunk + 1].

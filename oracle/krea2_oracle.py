@@ -480,16 +480,16 @@ def block_causal_allowed(ids: np.ndarray) -> np.ndarray:
 
 def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.ndarray, key_valid: np.ndarray,
                      scale: float) -> np.ndarray:
-    """GQA softmax attention where query row i of batch row b reads keys with
+    """GQA softmax attention where query row i of batch row b reads keys j with
     allowed[i, j] and key_valid[b, j]; a row with no readable key outputs zeros.
-    q (B, S, H, D); k, v (B, S, Hkv, D); allowed (S, S); key_valid (B, S). Returns fp64."""
-    B, S, H, D = q.shape
+    q (B, Sq, H, D); k, v (B, Sk, Hkv, D); allowed (Sq, Sk); key_valid (B, Sk). Returns fp64."""
+    B, Sq, H, D = q.shape
     G = H // k.shape[2]
-    out = np.zeros((B, S, H, D), dtype=np.float64)
+    out = np.zeros((B, Sq, H, D), dtype=np.float64)
     for b in range(B):
         for h in range(H):
             j = h // G
-            for i in range(S):
+            for i in range(Sq):
                 idx = np.nonzero(allowed[i] & key_valid[b])[0]
                 if idx.size == 0:
                     continue
@@ -497,3 +497,17 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, allowed: np.nd
                 p = np.exp(s - s.max())
                 out[b, i, h, :] = (p / p.sum()) @ v[b, idx, j, :].astype(np.float64)
     return out
+
+
+def cached_step_attention(q_new: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, k_new: np.ndarray,
+                          v_new: np.ndarray, allowed_new: np.ndarray, key_valid: np.ndarray,
+                          scale: float) -> np.ndarray:
+    """One denoising step of the block-causal variant with a key/value cache (page
+    "QwenImage21Transformer2DModel", kv_cache with causal_condition): the P prefix tokens are
+    not recomputed; their keys and values come from the cache, the Nq new tokens' own keys and
+    values follow them, and new token i reads the keys its row of the pattern allows.
+    q_new (B, Nq, H, D); k_cache, v_cache (B, P, Hkv, D); k_new, v_new (B, Nq, Hkv, D);
+    allowed_new (Nq, P + Nq), the pattern's rows of the new tokens; key_valid (B, P + Nq)."""
+    k = np.concatenate([k_cache, k_new], axis=1)
+    v = np.concatenate([v_cache, v_new], axis=1)
+    return masked_attention(q_new, k, v, allowed_new, key_valid, scale)

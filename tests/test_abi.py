@@ -100,3 +100,30 @@ def test_block_causal_key_end_matches_the_oracle_pattern(K2):
     bad = np.array([0, 0, -1, 0], dtype=np.int32)  # block 0 split in two runs
     with pytest.raises(K2.Krea2Error):
         K2.block_causal_key_end(bad)
+
+
+def test_kv_cache_argument_checks_on_host(K2):
+    # every rejection happens before anything is launched (the pointers are never touched)
+    d = K2.dims_struct(KI.FULL)
+    lib = K2.lib()
+    fake = 1 << 20
+    assert lib.krea2_kv_cache_attention_workspace_size(ctypes.byref(d), 2, 1024, K2.KREA2_BF16) == 2 * 1024 * 48 * 128 * 2
+    assert lib.krea2_kv_cache_attention_workspace_size(ctypes.byref(d), 2, 1024, K2.KREA2_F32) == 0
+    # rows [row0, row0 + n) must fit the capacity
+    rc = lib.krea2_kv_cache_append(ctypes.byref(d), 2, 100, 950, 1000, K2.KREA2_BF16, fake, fake, fake, fake, fake,
+                                   fake, None)
+    assert rc == -1 and b"capacity" in lib.krea2_last_error_string()
+    rc = lib.krea2_kv_cache_append(ctypes.byref(d), 2, 100, 0, 1000, K2.KREA2_F32, fake, fake, fake, fake, fake, fake,
+                                   None)
+    assert rc == -5
+    rc = lib.krea2_kv_cache_append(ctypes.byref(d), 2, 100, 0, 1000, K2.KREA2_BF16, fake, fake, fake, fake, fake + 8,
+                                   fake, None)
+    assert rc == -1 and b"aligned" in lib.krea2_last_error_string()
+    # the queries are the last Nq of L cached keys, and the cache must hold L rows
+    for T, L, Nq, cap in ((0, 100, 101, 200), (120, 100, 10, 200), (0, 300, 10, 200)):
+        rc = lib.krea2_gqa_attention_kv_cache(ctypes.byref(d), 2, T, L, Nq, K2.KREA2_BF16, fake, fake, fake, fake,
+                                              None, fake, fake, cap, None, fake, fake, 1 << 30, None)
+        assert rc == -1, (T, L, Nq, cap)
+    rc = lib.krea2_gqa_attention_kv_cache(ctypes.byref(d), 2, 0, 300, 10, K2.KREA2_BF16, fake, fake, fake, fake, None,
+                                          fake, fake, 300, None, fake, fake, 10, None)
+    assert rc == -2  # workspace too small

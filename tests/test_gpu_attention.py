@@ -162,3 +162,63 @@ def test_attention_block_causal(K2, segs, lengths):
     o = O.masked_attention(q, k, v, O.block_causal_allowed(ids), kv, 1.0 / np.sqrt(d.D))
     ref = o.reshape(B, S, d.HD) * O.sigmoid(g)
     assert rel_err(host(out).reshape(B, S, d.HD), ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("head,tail,lengths,spare", [
+    # the image being denoised after a cached prompt and condition image: every key readable
+    ([("text", 300), ("image", 256)], [("image", 1024)], [300, 77], 37),
+    # new text and image tokens after the cached prefix: per-token key_end of the pattern
+    ([("text", 100), ("image", 128)], [("text", 40), ("image", 200)], [100, 9], 0),
+])
+def test_attention_kv_cache(K2, head, tail, lengths, spare):
+    d = KI.FULL
+    ids = O.image_block_ids(head + tail)
+    S, P = len(ids), len(O.image_block_ids(head))
+    Nq, B = S - P, 2
+    cap = S + spare
+    last_text = int(np.nonzero(ids < 0)[0].max()) + 1
+    T = last_text if tail[0][0] == "image" else S  # keys [0, T) sit under the text mask
+    mask = np.ones((B, T), dtype=bool)
+    first_text = head[0][1]
+    for b, n in enumerate(lengths):
+        mask[b, n:first_text] = False  # the prompt is right-padded
+    kv = np.ones((B, S), dtype=bool)
+    kv[:, :T] = mask
+    x = KI.qkvg_raw(d, B, S, key=21)
+    w = KI.block_weights(d, 0)
+    pos = np.zeros((S, 3), dtype=np.float32)
+    pos[:, 1] = np.arange(S) // 32
+    pos[:, 2] = np.arange(S) % 32
+    cs = torch.empty(S, d.D // 2, device="cuda")
+    sn = torch.empty_like(cs)
+    K2.rope_tables(d, dev(pos, torch.float32), cs, sn)
+    xg = dev(x, torch.bfloat16).view(B, S, -1)
+    x_prefix = xg[:, :P].reshape(B * P, -1).contiguous()
+    x_new = xg[:, P:].reshape(B * Nq, -1).contiguous()
+    qw, kw = dev(w["q_norm_w"], torch.float32), dev(w["k_norm_w"], torch.float32)
+    # rows past L hold NaN: a read beyond the cached keys or across batch rows would show
+    kc = torch.full((B, cap, d.KVD), float("nan"), device="cuda", dtype=torch.bfloat16)
+    vc = torch.full_like(kc, float("nan"))
+    K2.kv_cache_append(d, B, P, 0, x_prefix, kw, cs[:P], sn[:P], kc, vc)
+    K2.kv_cache_append(d, B, Nq, P, x_new, kw, cs[P:], sn[P:], kc, vc)
+    key_end = None if tail == [("image", tail[0][1])] else dev(K2.block_causal_key_end(ids)[P:], torch.int32)
+    out = torch.empty(B * Nq, d.HD, device="cuda", dtype=torch.bfloat16)
+    ws = torch.empty(K2.kv_cache_attention_workspace_size(d, B, Nq, torch.bfloat16), dtype=torch.uint8, device="cuda")
+    K2.gqa_attention_kv_cache(d, B, T, S, Nq, x_new, qw, cs[P:], sn[P:], dev(mask.astype(np.uint8), torch.uint8),
+                              kc, vc, key_end, out, ws)
+    K2.check_device_error()
+
+    c, s = O.rope_cos_sin(pos, d.axes, d.theta)
+    xf = x.astype(np.float64).reshape(B, S, -1)
+    q = O.apply_rope(O.rms_norm(xf[..., :d.HD].reshape(B, S, d.H, d.D), w["q_norm_w"], d.eps), c, s)
+    k = O.apply_rope(O.rms_norm(xf[..., d.HD:d.HD + d.KVD].reshape(B, S, d.Hkv, d.D), w["k_norm_w"], d.eps), c, s)
+    v = xf[..., d.HD + d.KVD:d.HD + 2 * d.KVD].reshape(B, S, d.Hkv, d.D)
+    g = xf[:, P:, d.HD + 2 * d.KVD:]
+    # the cache: v is the projection copied bit for bit, k the normalised and rotated keys, spare rows untouched
+    assert torch.equal(vc[:, :S], xg[..., d.HD + d.KVD:d.HD + 2 * d.KVD])
+    assert rel_err(host(kc[:, :S]).reshape(B, S, d.Hkv, d.D), k, "k cache") < TOL_BF16
+    assert torch.isnan(kc[:, S:]).all() and torch.isnan(vc[:, S:]).all()
+    o = O.cached_step_attention(q[:, P:], k[:, :P], v[:, :P], k[:, P:], v[:, P:], O.block_causal_allowed(ids)[P:],
+                                kv, 1.0 / np.sqrt(d.D))
+    ref = o.reshape(B, Nq, d.HD) * O.sigmoid(g)
+    assert rel_err(host(out).reshape(B, Nq, d.HD), ref, "kv-cache attention") < TOL_BF16

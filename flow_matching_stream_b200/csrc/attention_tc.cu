@@ -134,8 +134,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   __shared__ __align__(8) uint64_t k_empty[KV_STAGES];  // freed when the S = Q K^T MMA is done
   __shared__ __align__(8) uint64_t v_empty[KV_STAGES];  // freed when the O += P V MMA is done
   __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t p_full;
-  __shared__ __align__(8) uint64_t pv_done;
+  // P_i is complete once all 256 softmax threads arrive on p_full[i & 1]. A fast warp may
+  // finish tile i+1 before a slow one finishes tile i (nothing else holds them together
+  // when no rescale waits on PV), so consecutive tiles count on different barriers; a warp
+  // cannot reach tile i+2 before PV_i, and so before every warp's arrival for tile i.
+  __shared__ __align__(8) uint64_t p_full[2];
+  __shared__ __align__(8) uint64_t pv_done[2];  // PV_i commits on pv_done[i & 1]
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -205,8 +209,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
-    mbar_init(&p_full, 256);
-    mbar_init(&pv_done, 1);
+    mbar_init(&p_full[0], 256);
+    mbar_init(&p_full[1], 256);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(&drain_bar, 1);
     for (int q = 0; q < 4; ++q) {
       mbar_init(&ex_bar[q], 64);
@@ -266,21 +272,26 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t sq = smem_u32(base + OFF_Q);
+      // Shared-memory descriptors differ only in the start-address field (bits 0..13, in
+      // 16-byte units), so each is a base descriptor plus a constant offset: the single issuing
+      // thread then spends almost no instructions between a barrier and its MMAs.
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(base + OFF_Q), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(base + OFF_K), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(base + OFF_V), KV_CHUNK, 1024);
       bool issued = false;
       auto issue_pv = [&](int i) -> bool {
         // O += P_i V_i : A = P_i in TMEM (bf16 pairs over its scores), B = V (MN-major)
         const int st = i % KV_STAGES;
-        if (!mbar_wait(&p_full, i & 1, abort)) return false;
+        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort)) return false;
         if (!mbar_wait(&v_full[st], (i / KV_STAGES) & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t sv = smem_u32(base + OFF_V + st * KV_TILE_BYTES);
+        const uint64_t dv = dv0 + (uint64_t)(st * (KV_TILE_BYTES >> 4));
         const uint32_t pt = tmem + (i & 1) * KT;
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk)
-          tc_mma_bf16_ts(tmem + O_COL, pt + kk * 8, smem_desc_sw128(sv + kk * 16 * 128, KV_CHUNK, 1024), IDESC_PV,
+          tc_mma_bf16_ts(tmem + O_COL, pt + kk * 8, dv + (uint64_t)(kk * 16 * 128 >> 4), IDESC_PV,
                          (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&pv_done);
+        tc_commit(&pv_done[i & 1]);
         tc_commit(&v_empty[st]);
         return true;
       };
@@ -289,14 +300,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           const int st = i % KV_STAGES;
           if (!mbar_wait(&k_full[st], (i / KV_STAGES) & 1, abort)) break;
           tc_fence_after();
-          const uint32_t sk = smem_u32(base + OFF_K + st * KV_TILE_BYTES);
+          const uint64_t dk = dk0 + (uint64_t)(st * (KV_TILE_BYTES >> 4));
           const uint32_t d_s = tmem + (i & 1) * KT;
 #pragma unroll
           for (int kk = 0; kk < AD / 16; ++kk) {
             const uint32_t qo = (kk >> 2) * Q_CHUNK + (kk & 3) * 32;
             const uint32_t ko = (kk >> 2) * KV_CHUNK + (kk & 3) * 32;
-            tc_mma_bf16(d_s, smem_desc_sw128(sq + qo, 16, 1024), smem_desc_sw128(sk + ko, 16, 1024), IDESC_QK,
-                        kk > 0 ? 1u : 0u);
+            tc_mma_bf16(d_s, dq0 + (uint64_t)(qo >> 4), dk + (uint64_t)(ko >> 4), IDESC_QK, kk > 0 ? 1u : 0u);
           }
           issued = true;
           tc_commit(&s_full[i & 1]);
@@ -388,11 +398,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       }
       l = l * alpha + rs;
       tmem_st16(sbase + half * (HK / 2), pk);  // P_i (bf16 pairs) over the tile's first 32 columns
-      if (i >= 1) {
-        // O must hold P_{i-1} V_{i-1} before it is rescaled (also keeps the phase count exact)
-        if (!mbar_wait(&pv_done, (i - 1) & 1, abort)) { ok = false; break; }
+      if (i >= 1 && any_grow) {
+        // O must hold P_{i-1} V_{i-1} before it is rescaled. PV_{i-1} is the ((i-1)/2)-th
+        // commit on pv_done[(i-1) & 1]; s_full_i already implies PV_{i-2} and earlier are
+        // done, and PV_{i+1} needs this tile's P, so the parity below names exactly that phase.
+        if (!mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        if (any_grow) {
+        {
 #pragma unroll 1
           for (int c = 0; c < AD / 64; ++c) {
             float o[32];
@@ -406,7 +418,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full);
+      mbar_arrive(&p_full[i & 1]);
     }
     const int pos = p0 + r % QPOS;
     const int h = j * G + r / QPOS;
@@ -419,7 +431,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       }
     } else if (ok) {
       // the output needs the last P V in O and both halves' row sums
-      ok = mbar_wait(&pv_done, (n - 1) & 1, abort);
+      ok = mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort);
       if (ok) {
         tc_fence_after();
         red_l[half][r] = l;

@@ -526,6 +526,11 @@ def time_attention_sweep(K2, torch, dev, steps: int, pk: dict) -> list:
     return out
 
 
+def kv_step_flops(d, Nq: int, valid_keys: int) -> float:
+    """Attention FLOPs of Nq new queries over the valid cached + new keys (per batch row)."""
+    return 4.0 * d.D * d.H * Nq * valid_keys
+
+
 def time_kv_cache_step(K2, torch, dev, steps: int, pk: dict) -> dict:
     """One denoising step's attention of the block-causal variant with a key/value cache: the
     prompt (512 text tokens, random valid length) and a 64x64 condition image are cached once;
@@ -569,7 +574,7 @@ def time_kv_cache_step(K2, torch, dev, steps: int, pk: dict) -> dict:
     torch.cuda.synchronize()
     K2.check_device_error()
     ms = e0.elapsed_time(e1) / steps
-    fl = 4.0 * d.D * d.H * Nq * (wl.lengths[0] + Ni + Nq)
+    fl = kv_step_flops(d, Nq, int(wl.lengths[0]) + Ni + Nq)
     return {"workload": "block-causal step with cached prompt + 64x64 condition image, 64x64 target",
             "new_tokens": Nq, "keys": L, "valid_text": int(wl.lengths[0]), "ms": ms,
             "tflops": fl / (ms / 1e3) / 1e12, "frac_burst": fl / (ms / 1e3) / 1e12 / pk["bf16_tflops"]}

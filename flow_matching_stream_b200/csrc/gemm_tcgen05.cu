@@ -14,7 +14,9 @@
 //               signals a finished accumulator.
 //   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane), reads 32 columns
 //               at a time with tcgen05.ld and applies the fused epilogue, while the MMA warp
-//               already accumulates the next tile into the other TMEM buffer.
+//               already accumulates the next tile into the other TMEM buffer. The residual
+//               epilogue transposes each 32x32 block through shared memory first, so that its
+//               fp32 read-modify-write of h runs in whole cache lines.
 // Tiles are visited in groups of row tiles (sized so the group's A tiles stay in L2) so that
 // concurrently running CTAs share W and A tiles through L2.
 #include <cuda.h>
@@ -41,7 +43,8 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN=256) or 16 KB (BN=128)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+  static constexpr int XPOSE_BYTES = 4 * 32 * 33 * 4;  // residual epilogue: one padded 32x32 fp32 tile per warp
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + XPOSE_BYTES + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 2 * BN;                         // double-buffered fp32
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 };
@@ -131,6 +134,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       int local = 0;
       bool issued = false;
+      // stage s's A tile starts s * STAGE_BYTES into the ring and its W tile A_BYTES later; a
+      // K step of 16 is 32 bytes: only the descriptor's start-address field (16-byte units)
+      // changes, so each MMA takes a base descriptor plus a constant
+      const uint64_t da0 = smem_desc_sw128(smem_u32(base), 16, 1024);
       for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
         const int acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
@@ -144,14 +151,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(base + stage * Cfg::STAGE_BYTES);
-          const uint32_t sb = sa + Cfg::A_BYTES;
+          const uint64_t ad = da0 + (uint64_t)(stage * (Cfg::STAGE_BYTES >> 4));
+          const uint64_t bd = ad + (uint64_t)(Cfg::A_BYTES >> 4);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = smem_desc_sw128(sa + k * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(sb + k * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, Cfg::IDESC, (kb | k) != 0);
-          }
+          for (int k = 0; k < BK / 16; ++k) tc_mma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, Cfg::IDESC, (kb | k) != 0);
           issued = true;
           tc_commit(&empty_bar[stage]);
           if (++stage == STAGES) {
@@ -308,27 +311,41 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       } else {  // EPI_RESID: h[row, col] += gate[b, col] * acc
-        float* hrow = reinterpret_cast<float*>(p.out) + (size_t)row * p.N + (size_t)nt * BN;
-        const int b = row_ok ? row / p.rows_per_batch : 0;
-        const float* grow = p.gate + (size_t)b * p.gate_stride + (size_t)nt * BN;
+        // After tcgen05.ld each thread holds one row of a 32-column chunk. Read-modify-write of
+        // the fp32 residual row by row would make every warp access touch 32 cache lines (one
+        // L1 wavefront each, in the SRAM that also feeds the tensor core), so the warp
+        // transposes its 32x32 block through a padded shared tile and then walks the rows: each
+        // access is one 128-byte line, and 16 rows of loads are in flight before any store.
+        float* xp = reinterpret_cast<float*>(base + STAGES * Cfg::STAGE_BYTES) + (warp - 2) * (32 * 33);
+        const int row0 = mt * BM + quarter * 32;
+        const int nrows = min(32, p.M - row0);
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
-          if (row_ok) {
-            float4* hp = reinterpret_cast<float4*>(hrow + c * 32);
-            const float4* gp = reinterpret_cast<const float4*>(grow + c * 32);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              float4 hv = hp[q];
-              const float4 gv = __ldg(gp + q);
-              hv.x += gv.x * v[q * 4 + 0];
-              hv.y += gv.y * v[q * 4 + 1];
-              hv.z += gv.z * v[q * 4 + 2];
-              hv.w += gv.w * v[q * 4 + 3];
-              hp[q] = hv;
+          for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = v[e];
+          __syncwarp();
+          const int col = nt * BN + c * 32 + lane;
+#pragma unroll 1
+          for (int i0 = 0; i0 < 32; i0 += 16) {
+            float* hp = reinterpret_cast<float*>(p.out) + (size_t)(row0 + i0) * p.N + col;
+            float hv[16];
+            {
+              const float* q = hp;
+#pragma unroll
+              for (int i = 0; i < 16; ++i, q += p.N) hv[i] = i0 + i < nrows ? *q : 0.f;
             }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int bb = (row0 + i0 + i) / p.rows_per_batch;
+              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i, hp += p.N)
+              if (i0 + i < nrows) *hp = hv[i];
           }
+          __syncwarp();
         }
       }
       tc_fence_before();

@@ -34,3 +34,11 @@ def test_norm_bytes():
     d = KI.FULL
     w = bench.block_kernel_work(d, 1, 512, 4096, [512])
     assert w["norm1"]["bytes"] == 4608 * 6144 * 6      # fp32 in, bf16 out
+
+
+def test_kv_cache_step_flops():
+    # 4096 target queries over 512 valid text + 4096 cached condition-image + 4096 own keys
+    d = KI.FULL
+    fl = bench.kv_step_flops(d, 4096, 512 + 4096 + 4096)
+    assert fl == 4 * 128 * 48 * 4096 * 8704
+    assert abs(fl / 1e12 - 0.8762) < 1e-3

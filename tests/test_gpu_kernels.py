@@ -57,7 +57,11 @@ def test_linear_swiglu(K2, M, F, K):
     assert rel_err(host(out), ref) < 8e-3
 
 
-@pytest.mark.parametrize("B,S,N,K", [(2, 150, 256, 512), (2, 4608, 6144, 16384)])
+@pytest.mark.parametrize("B,S,N,K", [
+    (2, 150, 256, 512),        # ragged rows; a batch boundary inside a 32-row block
+    (5, 20, 256, 128),         # one 32-row block spans three batch rows
+    (2, 4608, 6144, 16384),    # the backbone's down projection at the 1024^2 CFG shape
+])
 def test_linear_gated_residual(K2, B, S, N, K):
     M = B * S
     A, W = _bf((M, K), 6), _bf((N, K), 7, K ** -0.5)

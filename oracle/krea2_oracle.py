@@ -14,7 +14,10 @@ Sources (cited below by these short names):
   Transformer 架构全解": §二 I/O contract, §三 defaults and the head-split check,
   §四 module list and data flow, §四.2 TransformerBlock, §四.3 Attention, §四.4 RMSNorm,
   §四.5 TimestepEmbedding, §四.6 FinalLayer, §七 quick start.
-* [PIPE] page "Krea 2" (Krea2Pipeline docs): ``prepare_position_ids``.
+* [PIPE] page "Krea 2" (Krea2Pipeline docs): ``prepare_position_ids``, the scheduler shift,
+  guidance and the sampling loop.
+* page "QwenImage21Transformer2DModel": the block-causal attention pattern and the key/value
+  cache of that variant (cited by name where used).
 
 Precision: ``dtype=np.float64`` runs everything in fp64 (tiny config); ``np.float32``
 runs the projections in fp32 and every softmax in fp64 (full size). Softmax is always
@@ -23,8 +26,11 @@ an explicit normalised exponential over all valid keys of the row, never tiled.
 Readings where the pages are silent or garbled (the extraction of [ARCH] dropped the
 ``+``, ``=`` operators of its block pseudo-code) are marked READING below.
 
-Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` against
-closed forms, invariants, library routines or brute force. Agreement with the trained
+Parity status: every function here is pinned against closed forms, invariants, library
+routines or brute force: the block, backbone and their parts by ``tests/test_oracle_pins.py``,
+the sampler by ``tests/test_oracle_sampler.py``, text fusion by
+``tests/test_oracle_text_fusion.py``, and the block-causal pattern and cached step by
+``tests/test_oracle_block_causal.py``. Agreement with the trained
 Krea 2 model itself is *unpinned*: no weights or reference outputs are available, and
 the RoPE pairing convention (READING in ``apply_rope``) cannot be told apart from the
 rotate-half alternative by any invariant.

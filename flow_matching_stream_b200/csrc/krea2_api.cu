@@ -45,7 +45,7 @@ namespace {
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 // [ARCH] §三: sum(axes_dims_rope) == attention_head_dim, else ValueError; plus the limits of
-// this build's kernels.
+// this library's kernels.
 int check_dims(const Krea2Dims* d, int dtype) {
   if (!d) return set_error(KREA2_ERR_ARG, "dims is NULL");
   if (dtype != KREA2_BF16 && dtype != KREA2_F32) return set_error(KREA2_ERR_ARG, "unknown dtype %d", dtype);

@@ -50,7 +50,7 @@ enum {
   KREA2_ERR_WORKSPACE = -2,    /* workspace smaller than krea2_workspace_size()          */
   KREA2_ERR_CUDA = -3,         /* a CUDA launch or driver call failed                     */
   KREA2_ERR_TIMEOUT = -4,      /* a bounded device-side wait expired                      */
-  KREA2_ERR_UNSUPPORTED = -5   /* valid arguments this build has no kernel for            */
+  KREA2_ERR_UNSUPPORTED = -5   /* valid arguments the library has no kernel for           */
 };
 
 enum { KREA2_BF16 = 0, KREA2_F32 = 1 };

@@ -581,14 +581,15 @@ namespace {
 template <int G, bool PREFIX>
 int launch_attention_g(const AttnTcArgs& a, cudaStream_t stream) {
   constexpr int QPOS = 128 / G;
-  static bool attr_done = false;
-  if (!attr_done) {
+  static std::atomic<uint64_t> attr_done{0};
+  const uint64_t dev_bit = device_bit();
+  if (!(attr_done.load(std::memory_order_acquire) & dev_bit) || !dev_bit) {
     if (cudaFuncSetAttribute(attn_gqa_tc_kernel<G, PREFIX>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATT_SMEM) !=
             cudaSuccess ||
         cudaFuncSetAttribute(attn_gqa_tc_kernel<G, PREFIX>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(attention) failed");
-    attr_done = true;
+    attr_done.fetch_or(dev_bit, std::memory_order_release);
   }
   const int S = a.T + a.N;
   const int Sq = a.Sq > 0 ? a.Sq : S;

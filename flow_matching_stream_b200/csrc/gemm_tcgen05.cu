@@ -428,12 +428,13 @@ namespace {
 template <int BN, int EPI>
 int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
-  static bool attr_done = false;
+  static std::atomic<uint64_t> attr_done{0};
   auto kern = gemm_bf16_tcgen05_kernel<BN, EPI>;
-  if (!attr_done) {
+  const uint64_t dev_bit = device_bit();
+  if (!(attr_done.load(std::memory_order_acquire) & dev_bit) || !dev_bit) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess)
       return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(gemm) failed");
-    attr_done = true;
+    attr_done.fetch_or(dev_bit, std::memory_order_release);
   }
   CUtensorMap ta, tb;
   int rc = make_tmap_bf16_2d(&ta, A, p0.K, p0.M, p0.K, BK, BM);

@@ -1,5 +1,6 @@
 // Internal declarations shared by the library's translation units (not part of the ABI).
 #pragma once
+#include <atomic>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -12,6 +13,13 @@ enum { EPI_STORE = KREA2_EPI_STORE, EPI_SWIGLU = KREA2_EPI_SWIGLU, EPI_RESID = K
 
 // Records a message for krea2_last_error_string() and returns `code`.
 int set_error(int code, const char* fmt, ...);
+// Kernel attributes (the dynamic shared-memory opt-in) hold per device. Launchers keep one
+// bit per device ordinal to set them once per device; 0 (ordinals >= 64) means set every time.
+inline uint64_t device_bit() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return 0;
+  return 1ull << d;
+}
 int num_sms();
 // Counts kernel launches (krea2_launch_count); every launcher calls it once per launch.
 void count_launch();

@@ -14,9 +14,10 @@
 //               signals a finished accumulator.
 //   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane), reads 32 columns
 //               at a time with tcgen05.ld and applies the fused epilogue, while the MMA warp
-//               already accumulates the next tile into the other TMEM buffer. The residual
-//               epilogue transposes each 32x32 block through shared memory first, so that its
-//               fp32 read-modify-write of h runs in whole cache lines.
+//               already accumulates the next tile into the other TMEM buffer. The residual,
+//               plain and q/k/v/gate epilogues pass each warp's 32 rows through a padded
+//               shared tile, so that global accesses run in whole 128-byte row segments (the
+//               SwiGLU epilogue, with half the output bytes, measured no gain from it).
 // Tiles are visited in groups of row tiles (sized so the group's A tiles stay in L2) so that
 // concurrently running CTAs share W and A tiles through L2.
 #include <cuda.h>
@@ -61,6 +62,22 @@ struct TileMap {
     nt = local / gsize;
   }
 };
+
+// Each thread holds 32 consecutive bf16 pairs (64 columns) of its accumulator row. The warp
+// writes its 32 rows through a padded shared tile, so every global store covers 128 bytes of
+// one row instead of 16 bytes of each of 32 rows.
+__device__ __forceinline__ void store_bf16_rows(uint32_t* xp, const uint32_t* pk, __nv_bfloat16* dst0, size_t ld,
+                                                int nrows, int lane) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = pk[e];
+  __syncwarp();
+  uint32_t* d = reinterpret_cast<uint32_t*>(dst0) + lane;
+  const size_t ldw = ld / 2;  // row stride in bf16 pairs
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i)
+    if (i < nrows) d[(size_t)i * ldw] = xp[i * 33 + lane];
+  __syncwarp();
+}
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
@@ -189,16 +206,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool row_ok = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
 
+      const int row0 = mt * BM + quarter * 32;
+      const int nrows = min(32, p.M - row0);
+      uint32_t* xpk = reinterpret_cast<uint32_t*>(base + STAGES * Cfg::STAGE_BYTES) + (warp - 2) * (32 * 33);
       if constexpr (EPI == EPI_STORE) {
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + (size_t)nt * BN;
+        __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row0 * p.N + (size_t)nt * BN;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(tbase + c * 32, v);
+        for (int c = 0; c < BN / 64; ++c) {
+          float v[64];
+          tmem_ld64(tbase + c * 64, v);
           if (p.bias) {
-            const float4* bp = reinterpret_cast<const float4*>(p.bias + (size_t)nt * BN + c * 32);
+            const float4* bp = reinterpret_cast<const float4*>(p.bias + (size_t)nt * BN + c * 64);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
+            for (int q = 0; q < 16; ++q) {
               const float4 bv = __ldg(bp + q);
               v[q * 4 + 0] += bv.x;
               v[q * 4 + 1] += bv.y;
@@ -206,18 +226,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
               v[q * 4 + 3] += bv.w;
             }
           }
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
+          uint32_t pk[32];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 w;
-              w.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-              w.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-              w.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-              w.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-              dst[q] = w;
-            }
-          }
+          for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+          store_bf16_rows(xpk, pk, out0 + c * 64, p.N, nrows, lane);
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
         // interleaved 64-row groups: columns [128g, 128g+64) gate, [128g+64, 128g+128) up
@@ -250,7 +262,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       } else if constexpr (EPI == EPI_QKV) {
         // [q | k | v | gate] columns; 128-wide q/k heads get RMSNorm (1 + w) and RoPE here,
         // once per element, on the fp32 accumulator (page §四.3 order: norm, then RoPE)
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * p.N + (size_t)nt * BN;
+        __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row0 * p.N + (size_t)nt * BN;
         const int pos = row_ok ? row % p.rows_per_batch : 0;
         const float* cs = p.cos + (size_t)pos * 64;
         const float* sn = p.sin + (size_t)pos * 64;
@@ -296,18 +308,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
                 }
               }
             }
-            if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + u * 128 + h2 * 64);
+            uint32_t pk[32];
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                uint4 w4o;
-                w4o.x = pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]);
-                w4o.y = pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]);
-                w4o.z = pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]);
-                w4o.w = pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]);
-                dst[q] = w4o;
-              }
-            }
+            for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+            store_bf16_rows(xpk, pk, out0 + u * 128 + h2 * 64, p.N, nrows, lane);
           }
         }
       } else {  // EPI_RESID: h[row, col] += gate[b, col] * acc
@@ -316,9 +320,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // L1 wavefront each, in the SRAM that also feeds the tensor core), so the warp
         // transposes its 32x32 block through a padded shared tile and then walks the rows: each
         // access is one 128-byte line, and 16 rows of loads are in flight before any store.
-        float* xp = reinterpret_cast<float*>(base + STAGES * Cfg::STAGE_BYTES) + (warp - 2) * (32 * 33);
-        const int row0 = mt * BM + quarter * 32;
-        const int nrows = min(32, p.M - row0);
+        float* xp = reinterpret_cast<float*>(xpk);
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];

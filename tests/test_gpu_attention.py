@@ -80,6 +80,19 @@ def test_attention_bf16_random_non_prefix_mask(K2):
     assert rel_err(out, ref) < TOL_BF16
 
 
+@pytest.mark.parametrize("seed,p_keep", [(3, 0.05), (4, 0.5), (5, 0.9), (6, 0.02)])
+def test_attention_bf16_masks_that_split_the_lane_quarters(K2, seed, p_keep):
+    # sparse random text masks make the running maxima of different rows grow on different
+    # tiles, so some lane quarters rescale O and others do not; the barrier protocol between
+    # the softmax warps and the MMA issuer must keep the result exact regardless
+    d = KI.FULL
+    B, T, gh, gw = 2, 320, 10, 12
+    mask = KI.random_keep_mask(B, T, p_keep, key=seed)
+    x, w, pos, out = run_attention(K2, d, B, T, gh, gw, mask, torch.bfloat16, key=seed)
+    ref = oracle_attention(d, x, w, pos, B, T, gh * gw, mask)
+    assert rel_err(out, ref, f"mask seed {seed} keep {p_keep}") < TOL_BF16
+
+
 def test_attention_bf16_padded_keys_are_ignored(K2):
     # changing padded text k/v in the raw projection must not change any output row
     d = KI.FULL

@@ -51,13 +51,14 @@ int check_dims(const Krea2Dims* d, int dtype) {
   if (dtype != KREA2_BF16 && dtype != KREA2_F32) return set_error(KREA2_ERR_ARG, "unknown dtype %d", dtype);
   if (d->H <= 0 || d->Hkv <= 0 || d->D <= 0 || d->C <= 0 || d->F <= 0)
     return set_error(KREA2_ERR_ARG, "non-positive model dimension");
-  if (d->C != d->H * d->D) return set_error(KREA2_ERR_ARG, "hidden size C=%d != heads*head_dim=%d", d->C, d->H * d->D);
+  if ((long long)d->C != (long long)d->H * d->D)
+    return set_error(KREA2_ERR_ARG, "hidden size C=%d != heads*head_dim=%lld", d->C, (long long)d->H * d->D);
   if (d->H % d->Hkv) return set_error(KREA2_ERR_ARG, "heads %d not a multiple of kv heads %d", d->H, d->Hkv);
   for (int a = 0; a < 3; ++a)
     if (d->axes[a] < 0 || (d->axes[a] & 1)) return set_error(KREA2_ERR_ARG, "RoPE axis %d has odd size %d", a, d->axes[a]);
-  if (d->axes[0] + d->axes[1] + d->axes[2] != d->D)
-    return set_error(KREA2_ERR_ARG, "sum(axes_dims_rope)=%d != attention_head_dim=%d",
-                     d->axes[0] + d->axes[1] + d->axes[2], d->D);
+  const long long axes_sum = (long long)d->axes[0] + d->axes[1] + d->axes[2];
+  if (axes_sum != d->D)
+    return set_error(KREA2_ERR_ARG, "sum(axes_dims_rope)=%lld != attention_head_dim=%d", axes_sum, d->D);
   if (!(d->theta > 0.f) || !(d->eps > 0.f)) return set_error(KREA2_ERR_ARG, "theta and eps must be positive");
   if (d->D != 64 && d->D != 128) return set_error(KREA2_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (d->C % 128 || d->C > 8192) return set_error(KREA2_ERR_UNSUPPORTED, "hidden size must be a multiple of 128, <= 8192");
@@ -78,7 +79,7 @@ int check_shape(int B, int T, int N) {
   if (B <= 0) return set_error(KREA2_ERR_ARG, "batch must be positive");
   if (T < 0) return set_error(KREA2_ERR_ARG, "text length must be >= 0");
   if (N <= 0) return set_error(KREA2_ERR_ARG, "image_seq_len must be >= 1 (every query then has a valid key)");
-  if ((long long)B * (T + N) > (1LL << 30)) return set_error(KREA2_ERR_ARG, "too many tokens");
+  if ((long long)B * ((long long)T + N) > (1LL << 30)) return set_error(KREA2_ERR_ARG, "too many tokens");
   return KREA2_OK;
 }
 
@@ -140,7 +141,7 @@ int attention_raw(const AttnParams& p, int dtype, void* ws, cudaStream_t s, cons
 
 size_t attention_ws_bytes(const Krea2Dims* d, int B, int T, int N, int dtype) {
   if (dtype == KREA2_BF16 && attention_tc_supported(d->D, d->H, d->Hkv))
-    return (size_t)B * (T + N) * (size_t)(d->H + d->Hkv) * d->D * 2;
+    return (size_t)B * ((size_t)T + N) * (size_t)(d->H + d->Hkv) * d->D * 2;
   return 0;
 }
 
@@ -332,7 +333,8 @@ int krea2_gqa_attention_block_causal(const Krea2Dims* dims, int B, int T, int N,
   if (rc) return rc;
   // every query reads at least its own position, so (unlike the plain entry) no image token is
   // needed; a query whose readable keys are all padded outputs zeros
-  if (B <= 0 || T < 0 || N < 0 || T + N <= 0) return set_error(KREA2_ERR_ARG, "need B >= 1 and T + N >= 1");
+  if (B <= 0 || T < 0 || N < 0 || (long long)T + N <= 0 || (long long)B * ((long long)T + N) > (1LL << 30))
+    return set_error(KREA2_ERR_ARG, "need B >= 1, T + N >= 1 and B * (T + N) <= 2^30");
   if (!qkvg || !q_norm_w || !k_norm_w || !cos || !sin || !out || !key_end)
     return set_error(KREA2_ERR_ARG, "NULL pointer");
   if (dtype != KREA2_BF16 || !attention_tc_supported(dims->D, dims->H, dims->Hkv))

@@ -127,3 +127,19 @@ def test_kv_cache_argument_checks_on_host(K2):
     rc = lib.krea2_gqa_attention_kv_cache(ctypes.byref(d), 2, 0, 300, 10, K2.KREA2_BF16, fake, fake, fake, fake, None,
                                           fake, fake, 300, None, fake, fake, 10, None)
     assert rc == -2  # workspace too small
+
+
+def test_token_counts_that_overflow_int_are_rejected(K2):
+    # T + N beyond 2^31 must be caught by the size checks, not wrap around
+    d = K2.dims_struct(KI.FULL)
+    lib = K2.lib()
+    big = (1 << 31) - 10
+    assert lib.krea2_workspace_size(ctypes.byref(d), 1, big, 100, K2.KREA2_BF16) == 0
+    assert lib.krea2_attention_workspace_size(ctypes.byref(d), 1, big, 100, K2.KREA2_BF16) == 0
+    fake = 1 << 20
+    rc = lib.krea2_gqa_attention_block_causal(ctypes.byref(d), 1, big, 100, K2.KREA2_BF16, fake, fake, fake, fake,
+                                              fake, None, fake, fake, fake, 1 << 40, None)
+    assert rc == -1 and b"2^30" in lib.krea2_last_error_string()
+    bad = K2.dims_struct(KI.FULL)
+    bad.H = 1 << 30                       # H * D overflows int
+    assert lib.krea2_workspace_size(ctypes.byref(bad), 1, 8, 8, K2.KREA2_BF16) == 0

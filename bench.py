@@ -253,6 +253,17 @@ def replica_throughput(world: int, steps: int, flops_per_step: float, ms_max: fl
     return world * steps * flops_per_step / (ms_max / 1e3) / 1e12
 
 
+def workload_config(wl: KI.Workload, world: int) -> dict:
+    """The `config` object both arms print for the backbone workload."""
+    d = wl.dims
+    return {"workload": wl.name, "batch": wl.B, "text_tokens": wl.T, "image_tokens": wl.N, "seq_len": wl.S,
+            "layers": d.n_layers, "hidden": d.C, "heads": f"{d.H}q/{d.Hkv}kv x {d.D}", "intermediate": d.F,
+            "weights": "random-init N(0,1)/sqrt(fan_in), seeded, ~12.2 B params bf16",
+            "l2": "inputs larger than L2: 24 GB of block weights stream from HBM every step",
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "flops_per_step": backbone_flops(d, wl.B, wl.T, wl.N, wl.lengths)}
+
+
 # ----------------------------------------------------------------------------- native arm
 
 def run_native(args, rank: int, world: int, local_rank: int) -> None:
@@ -366,12 +377,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": B, "text_tokens": T, "image_tokens": N, "seq_len": S,
-                   "layers": d.n_layers, "hidden": d.C, "heads": f"{d.H}q/{d.Hkv}kv x {d.D}",
-                   "intermediate": d.F, "weights": "random-init N(0,1)/sqrt(fan_in), seeded, ~12.2 B params bf16",
-                   "l2": "inputs larger than L2: 24 GB of block weights stream from HBM every step",
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "flops_per_step": flops_step},
+        "config": workload_config(wl, world),
         "backbone_ms_per_step": ms_step,
         "sampler_1024sq": sampler,
         "text_fusion_once_per_prompt": text,
@@ -668,8 +674,7 @@ def run_reference(args, rank: int) -> None:
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "batch": wl.B, "text_tokens": wl.T, "image_tokens": wl.N,
-                       "layers": wl.dims.n_layers},
+            "config": workload_config(wl, args.gpus),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
                              "kind": "oracle", "sample": o.describe(el / args.steps)},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

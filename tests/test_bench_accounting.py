@@ -42,3 +42,11 @@ def test_kv_cache_step_flops():
     fl = bench.kv_step_flops(d, 4096, 512 + 4096 + 4096)
     assert fl == 4 * 128 * 48 * 4096 * 8704
     assert abs(fl / 1e12 - 0.8762) < 1e-3
+
+
+def test_both_arms_print_the_same_config():
+    wl = KI.backbone_1024()
+    c = bench.workload_config(wl, 1)
+    assert c["workload"] == wl.name and c["seq_len"] == 4608 and c["layers"] == 28
+    assert abs(c["flops_per_step"] / 1e12 - 126.64) < 0.01
+    assert c["parallelism"] == "single GPU" and bench.workload_config(wl, 8)["parallelism"] == "replicas"

@@ -1,0 +1,205 @@
+"""A randomized model check of the attention kernel's barrier protocol (CPU).
+
+The tensor-core attention kernel (attention_tc.cu) coordinates one MMA-issuing thread, the
+tensor pipe and eight softmax warps (two per TMEM lane quarter) through mbarriers:
+
+* ``s_full[i & 1]``: committed after S_i = Q K_i^T;
+* ``p_full[i & 1]``: all softmax warps wrote P_i over their scores;
+* ``pv_done[i & 1]``: committed after O += P_i V_i;
+* ``ex_bar[q]``: the two halves of lane quarter q exchanged their row maxima.
+
+This file restates those roles as Python generators and runs them under many random
+interleavings. An mbarrier wait on parity P passes when the number of completed phases has the
+other parity, exactly the hardware's rule, so a barrier that runs two phases ahead of a waiter
+is mistaken for one that has not completed: the model reproduces that aliasing. The tensor
+pipe executes issued MMAs in order, and a commit arrives once everything issued before it has
+run. Checked invariants:
+
+* P·V for tile i runs only after every warp wrote its part of P_i;
+* a score buffer is overwritten by QK^T only after the P·V that read its P;
+* a warp reads S_i while the buffer still holds S_i, and the partner's row max of tile i;
+* O is rescaled only between P·V_{i-1} and P·V_i;
+* at the end every P·V has run, in order.
+
+Two negative controls must fail: the same model with a single p_full barrier (the protocol
+before consecutive tiles were split across two barriers), and one whose softmax warps skip
+the max exchange.
+"""
+import random
+
+import pytest
+
+N_QUARTERS, N_HALVES = 4, 2
+N_WARPS = N_QUARTERS * N_HALVES
+
+
+class Barrier:
+    def __init__(self, count: int):
+        self.count, self.arrived, self.completed = count, 0, 0
+
+    def arrive(self):
+        self.arrived += 1
+        if self.arrived == self.count:
+            self.arrived = 0
+            self.completed += 1
+
+    def test_parity(self, parity: int) -> bool:
+        # mbarrier.try_wait.parity: passes once the phase of that parity has completed, i.e.
+        # while the current (incomplete) phase has the other parity
+        return (self.completed & 1) != parity
+
+
+class Violation(AssertionError):
+    pass
+
+
+class Model:
+    def __init__(self, n_tiles: int, grows, split_p_full: bool, exchange: bool = True):
+        self.n = n_tiles
+        self.grows = grows  # grows[(quarter, tile)]: the quarter's rows rescale O at that tile
+        self.s_full = [Barrier(1), Barrier(1)]
+        self.pv_done = [Barrier(1), Barrier(1)]
+        nb = 2 if split_p_full else 1
+        self.p_full = [Barrier(N_WARPS) for _ in range(nb)]
+        self.split = split_p_full
+        self.exchange = exchange          # False: a warp does not wait for its partner's max
+        self.ex_bar = [Barrier(N_HALVES) for _ in range(N_QUARTERS)]
+        self.fifo = []                    # issued tensor-pipe work, executed in order
+        self.s_buf = [None, None]         # tile whose scores (or P) the buffer holds
+        self.p_written = [dict(), dict()]  # buffer -> {(q, h): tile}
+        self.pv_applied = []              # tiles whose P·V ran, in order
+        self.red_max = {}                 # (parity, q, h) -> tile
+        self.read_scores = set()          # (tile, q, h): that half has read its scores
+
+    def pfull(self, i):
+        return self.p_full[i & 1] if self.split else self.p_full[0]
+
+    def pfull_parity(self, i):
+        return ((i >> 1) & 1) if self.split else (i & 1)
+
+    # ---- roles -------------------------------------------------------------------------
+    def mma_thread(self):
+        def issue_pv(i):
+            while not self.pfull(i).test_parity(self.pfull_parity(i)):
+                yield
+            self.fifo.append(("PV", i))
+            self.fifo.append(("COMMIT", self.pv_done[i & 1]))
+            yield
+
+        for i in range(self.n):
+            self.fifo.append(("QK", i))
+            self.fifo.append(("COMMIT", self.s_full[i & 1]))
+            yield
+            if i >= 1:
+                yield from issue_pv(i - 1)
+        if self.n:
+            yield from issue_pv(self.n - 1)
+
+    def tensor_pipe(self):
+        while True:
+            if not self.fifo:
+                yield
+                continue
+            op = self.fifo.pop(0)
+            if op[0] == "QK":
+                i = op[1]
+                if i >= 2 and (i - 2) not in self.pv_applied:
+                    raise Violation(f"QK_{i} overwrote the score buffer before PV_{i - 2} read it")
+                self.s_buf[i & 1] = i
+            elif op[0] == "PV":
+                i = op[1]
+                written = self.p_written[i & 1]
+                missing = [k for k in written if written[k] != i] + \
+                          [(q, h) for q in range(N_QUARTERS) for h in range(N_HALVES) if (q, h) not in written]
+                if missing:
+                    raise Violation(f"PV_{i} ran before P_{i} was written by warps {sorted(set(missing))}")
+                if self.pv_applied != list(range(i)):
+                    raise Violation(f"PV_{i} ran out of order after {self.pv_applied}")
+                self.pv_applied.append(i)
+            else:
+                op[1].arrive()
+            yield
+
+    def softmax_warp(self, q: int, h: int):
+        for i in range(self.n):
+            while not self.s_full[i & 1].test_parity((i >> 1) & 1):
+                yield
+            if self.s_buf[i & 1] != i:
+                raise Violation(f"warp ({q},{h}) read buffer {i & 1} holding tile {self.s_buf[i & 1]}, not {i}")
+            self.read_scores.add((i, q, h))
+            self.red_max[(i & 1, q, h)] = i
+            self.ex_bar[q].arrive()
+            yield
+            while self.exchange and not self.ex_bar[q].test_parity(i & 1):
+                yield
+            if self.red_max.get((i & 1, q, 1 - h)) != i:
+                raise Violation(f"warp ({q},{h}) read its partner's max of tile {self.red_max.get((i & 1, q, 1 - h))}")
+            if (i, q, 1 - h) not in self.read_scores:
+                raise Violation(f"warp ({q},{h}) wrote P_{i} before its partner read the scores under it")
+            self.p_written[i & 1][(q, h)] = i
+            yield
+            if i >= 1 and self.grows[(q, i)]:
+                b = self.pv_done[(i - 1) & 1]
+                while not b.test_parity(((i - 1) >> 1) & 1):
+                    yield
+                if (i - 1) not in self.pv_applied or i in self.pv_applied:
+                    raise Violation(f"warp ({q},{h}) rescaled O at tile {i} with P·V done for {self.pv_applied}")
+            self.pfull(i).arrive()
+            yield
+        if self.n:
+            b = self.pv_done[(self.n - 1) & 1]
+            while not b.test_parity(((self.n - 1) >> 1) & 1):
+                yield
+            if self.pv_applied != list(range(self.n)):
+                raise Violation(f"warp ({q},{h}) read O with P·V done for {self.pv_applied}")
+
+
+def run(n_tiles: int, seed: int, split_p_full: bool = True, exchange: bool = True, max_steps: int = 200_000):
+    rng = random.Random(seed)
+    grows = {(q, i): rng.random() < 0.3 for q in range(N_QUARTERS) for i in range(n_tiles)}
+    m = Model(n_tiles, grows, split_p_full, exchange)
+    roles = [m.mma_thread()] + [m.softmax_warp(q, h) for q in range(N_QUARTERS) for h in range(N_HALVES)]
+    pipe = m.tensor_pipe()
+    live = list(range(len(roles)))
+    # a skewed speed per role makes one quarter run well ahead of another
+    speed = [rng.choice((1, 1, 2, 8)) for _ in roles]
+    for _ in range(max_steps):
+        if not live:
+            return m
+        if rng.random() < 0.3:
+            next(pipe)
+            continue
+        k = rng.choices(live, weights=[speed[j] for j in live])[0]
+        try:
+            next(roles[k])
+        except StopIteration:
+            live.remove(k)
+    raise Violation(f"no progress after {max_steps} steps (roles left: {live})")
+
+
+@pytest.mark.parametrize("n_tiles", [1, 2, 3, 7])
+def test_protocol_holds_under_random_interleavings(n_tiles):
+    for seed in range(300):
+        m = run(n_tiles, seed)
+        assert m.pv_applied == list(range(n_tiles))
+
+
+def test_a_single_p_full_barrier_lets_a_fast_quarter_complete_a_slow_quarters_phase():
+    failures = 0
+    for seed in range(400):
+        try:
+            run(6, seed, split_p_full=False)
+        except Violation:
+            failures += 1
+    assert failures > 0
+
+
+def test_writing_p_without_the_max_exchange_is_caught():
+    # the exchange is also what keeps half 1's P off half 0's unread scores
+    failures = 0
+    for seed in range(200):
+        try:
+            run(4, seed, exchange=False)
+        except Violation:
+            failures += 1
+    assert failures > 0

@@ -29,28 +29,10 @@ import random
 
 import pytest
 
+from protocol_model import Barrier, Violation, schedule
+
 N_QUARTERS, N_HALVES = 4, 2
 N_WARPS = N_QUARTERS * N_HALVES
-
-
-class Barrier:
-    def __init__(self, count: int):
-        self.count, self.arrived, self.completed = count, 0, 0
-
-    def arrive(self):
-        self.arrived += 1
-        if self.arrived == self.count:
-            self.arrived = 0
-            self.completed += 1
-
-    def test_parity(self, parity: int) -> bool:
-        # mbarrier.try_wait.parity: passes once the phase of that parity has completed, i.e.
-        # while the current (incomplete) phase has the other parity
-        return (self.completed & 1) != parity
-
-
-class Violation(AssertionError):
-    pass
 
 
 class Model:
@@ -159,22 +141,8 @@ def run(n_tiles: int, seed: int, split_p_full: bool = True, exchange: bool = Tru
     grows = {(q, i): rng.random() < 0.3 for q in range(N_QUARTERS) for i in range(n_tiles)}
     m = Model(n_tiles, grows, split_p_full, exchange)
     roles = [m.mma_thread()] + [m.softmax_warp(q, h) for q in range(N_QUARTERS) for h in range(N_HALVES)]
-    pipe = m.tensor_pipe()
-    live = list(range(len(roles)))
-    # a skewed speed per role makes one quarter run well ahead of another
-    speed = [rng.choice((1, 1, 2, 8)) for _ in roles]
-    for _ in range(max_steps):
-        if not live:
-            return m
-        if rng.random() < 0.3:
-            next(pipe)
-            continue
-        k = rng.choices(live, weights=[speed[j] for j in live])[0]
-        try:
-            next(roles[k])
-        except StopIteration:
-            live.remove(k)
-    raise Violation(f"no progress after {max_steps} steps (roles left: {live})")
+    schedule(rng, roles, [m.tensor_pipe()], max_steps)
+    return m
 
 
 @pytest.mark.parametrize("n_tiles", [1, 2, 3, 7])

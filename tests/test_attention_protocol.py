@@ -6,7 +6,9 @@ tensor pipe and eight softmax warps (two per TMEM lane quarter) through mbarrier
 * ``s_full[i & 1]``: committed after S_i = Q K_i^T;
 * ``p_full[i & 1]``: all softmax warps wrote P_i over their scores;
 * ``pv_done[i & 1]``: committed after O += P_i V_i;
-* ``ex_bar[q]``: the two halves of lane quarter q exchanged their row maxima.
+* ``ex_bar[q]``: the two halves of lane quarter q exchanged their row maxima;
+* ``k_full``/``k_empty`` and ``v_full``/``v_empty``: the two-stage K and V rings the TMA
+  producer fills (K tile i+1 is loaded before V tile i).
 
 This file restates those roles as Python generators and runs them under many random
 interleavings. An mbarrier wait on parity P passes when the number of completed phases has the
@@ -16,14 +18,16 @@ pipe executes issued MMAs in order, and a commit arrives once everything issued 
 run. Checked invariants:
 
 * P·V for tile i runs only after every warp wrote its part of P_i;
+* QK^T and P·V read K and V stages that hold their tile, and no load overwrites a stage
+  before the MMA that reads it has run;
 * a score buffer is overwritten by QK^T only after the P·V that read its P;
 * a warp reads S_i while the buffer still holds S_i, and the partner's row max of tile i;
 * O is rescaled only between P·V_{i-1} and P·V_i;
 * at the end every P·V has run, in order.
 
-Two negative controls must fail: the same model with a single p_full barrier (the protocol
-before consecutive tiles were split across two barriers), and one whose softmax warps skip
-the max exchange.
+Three negative controls must fail: the same model with a single p_full barrier (the protocol
+before consecutive tiles were split across two barriers), one whose softmax warps skip the max
+exchange, and one that frees V stages after QK^T instead of after P·V.
 """
 import random
 
@@ -33,10 +37,11 @@ from protocol_model import Barrier, Violation, schedule
 
 N_QUARTERS, N_HALVES = 4, 2
 N_WARPS = N_QUARTERS * N_HALVES
+KV_STAGES = 2
 
 
 class Model:
-    def __init__(self, n_tiles: int, grows, split_p_full: bool, exchange: bool = True):
+    def __init__(self, n_tiles: int, grows, split_p_full: bool, exchange: bool = True, early_v_release: bool = False):
         self.n = n_tiles
         self.grows = grows  # grows[(quarter, tile)]: the quarter's rows rescale O at that tile
         self.s_full = [Barrier(1), Barrier(1)]
@@ -45,6 +50,7 @@ class Model:
         self.p_full = [Barrier(N_WARPS) for _ in range(nb)]
         self.split = split_p_full
         self.exchange = exchange          # False: a warp does not wait for its partner's max
+        self.early_v_release = early_v_release  # True: V stages freed after QK^T, not after P·V
         self.ex_bar = [Barrier(N_HALVES) for _ in range(N_QUARTERS)]
         self.fifo = []                    # issued tensor-pipe work, executed in order
         self.s_buf = [None, None]         # tile whose scores (or P) the buffer holds
@@ -52,6 +58,15 @@ class Model:
         self.pv_applied = []              # tiles whose P·V ran, in order
         self.red_max = {}                 # (parity, q, h) -> tile
         self.read_scores = set()          # (tile, q, h): that half has read its scores
+        # K/V rings of KV_STAGES stages each, filled by the TMA producer
+        self.k_full = [Barrier(1) for _ in range(KV_STAGES)]
+        self.v_full = [Barrier(1) for _ in range(KV_STAGES)]
+        self.k_empty = [Barrier(1) for _ in range(KV_STAGES)]
+        self.v_empty = [Barrier(1) for _ in range(KV_STAGES)]
+        self.k_stage = [None] * KV_STAGES  # tile whose K the stage holds
+        self.v_stage = [None] * KV_STAGES
+        self.tma = []                      # in-flight loads: ("K" | "V", stage, tile)
+        self.qk_done = set()
 
     def pfull(self, i):
         return self.p_full[i & 1] if self.split else self.p_full[0]
@@ -62,20 +77,65 @@ class Model:
     # ---- roles -------------------------------------------------------------------------
     def mma_thread(self):
         def issue_pv(i):
+            st = i % KV_STAGES
             while not self.pfull(i).test_parity(self.pfull_parity(i)):
+                yield
+            while not self.v_full[st].test_parity((i // KV_STAGES) & 1):
                 yield
             self.fifo.append(("PV", i))
             self.fifo.append(("COMMIT", self.pv_done[i & 1]))
+            if not self.early_v_release:
+                self.fifo.append(("COMMIT", self.v_empty[st]))
             yield
 
         for i in range(self.n):
+            st = i % KV_STAGES
+            while not self.k_full[st].test_parity((i // KV_STAGES) & 1):
+                yield
             self.fifo.append(("QK", i))
             self.fifo.append(("COMMIT", self.s_full[i & 1]))
+            self.fifo.append(("COMMIT", self.k_empty[st]))
+            if self.early_v_release:
+                self.fifo.append(("COMMIT", self.v_empty[st]))
             yield
             if i >= 1:
                 yield from issue_pv(i - 1)
         if self.n:
             yield from issue_pv(self.n - 1)
+
+    def producer(self):
+        # K tile i+1 is issued before V tile i: K stages free up after QK^T, V stages only
+        # after P·V, so the K loads run a tile further ahead
+        def load(kind, i):
+            st = i % KV_STAGES
+            empty = self.k_empty if kind == "K" else self.v_empty
+            while not empty[st].test_parity(((i // KV_STAGES) & 1) ^ 1):
+                yield
+            self.tma.append((kind, st, i))
+            yield
+
+        if self.n:
+            yield from load("K", 0)
+        for i in range(self.n):
+            if i + 1 < self.n:
+                yield from load("K", i + 1)
+            yield from load("V", i)
+
+    def tma_engine(self):
+        while True:
+            if self.tma:
+                kind, st, i = self.tma.pop(0)
+                if kind == "K":
+                    if i >= KV_STAGES and (i - KV_STAGES) not in self.qk_done:
+                        raise Violation(f"K_{i} overwrote stage {st} before QK_{i - KV_STAGES} read it")
+                    self.k_stage[st] = i
+                    self.k_full[st].arrive()
+                else:
+                    if i >= KV_STAGES and (i - KV_STAGES) not in self.pv_applied:
+                        raise Violation(f"V_{i} overwrote stage {st} before PV_{i - KV_STAGES} read it")
+                    self.v_stage[st] = i
+                    self.v_full[st].arrive()
+            yield
 
     def tensor_pipe(self):
         while True:
@@ -87,7 +147,10 @@ class Model:
                 i = op[1]
                 if i >= 2 and (i - 2) not in self.pv_applied:
                     raise Violation(f"QK_{i} overwrote the score buffer before PV_{i - 2} read it")
+                if self.k_stage[i % KV_STAGES] != i:
+                    raise Violation(f"QK_{i} read K stage holding tile {self.k_stage[i % KV_STAGES]}")
                 self.s_buf[i & 1] = i
+                self.qk_done.add(i)
             elif op[0] == "PV":
                 i = op[1]
                 written = self.p_written[i & 1]
@@ -97,6 +160,8 @@ class Model:
                     raise Violation(f"PV_{i} ran before P_{i} was written by warps {sorted(set(missing))}")
                 if self.pv_applied != list(range(i)):
                     raise Violation(f"PV_{i} ran out of order after {self.pv_applied}")
+                if self.v_stage[i % KV_STAGES] != i:
+                    raise Violation(f"PV_{i} read V stage holding tile {self.v_stage[i % KV_STAGES]}")
                 self.pv_applied.append(i)
             else:
                 op[1].arrive()
@@ -136,12 +201,14 @@ class Model:
                 raise Violation(f"warp ({q},{h}) read O with P·V done for {self.pv_applied}")
 
 
-def run(n_tiles: int, seed: int, split_p_full: bool = True, exchange: bool = True, max_steps: int = 200_000):
+def run(n_tiles: int, seed: int, split_p_full: bool = True, exchange: bool = True, early_v_release: bool = False,
+        max_steps: int = 200_000):
     rng = random.Random(seed)
     grows = {(q, i): rng.random() < 0.3 for q in range(N_QUARTERS) for i in range(n_tiles)}
-    m = Model(n_tiles, grows, split_p_full, exchange)
-    roles = [m.mma_thread()] + [m.softmax_warp(q, h) for q in range(N_QUARTERS) for h in range(N_HALVES)]
-    schedule(rng, roles, [m.tensor_pipe()], max_steps)
+    m = Model(n_tiles, grows, split_p_full, exchange, early_v_release)
+    roles = [m.producer(), m.mma_thread()] + [m.softmax_warp(q, h) for q in range(N_QUARTERS)
+                                              for h in range(N_HALVES)]
+    schedule(rng, roles, [m.tensor_pipe(), m.tma_engine()], max_steps)
     return m
 
 
@@ -171,3 +238,12 @@ def test_writing_p_without_the_max_exchange_is_caught():
         except Violation:
             failures += 1
     assert failures > 0
+
+
+def test_releasing_v_stages_before_p_v_is_caught():
+    for seed in range(200):
+        try:
+            run(6, seed, early_v_release=True, max_steps=50_000)
+        except Violation:
+            return
+    pytest.fail("early V release passed every interleaving")

@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         for (int c = 0; c < 2; ++c)
           tma_load_3d(base + OFF_Q + c * Q_CHUNK + hl * (QPOS * 128), &tmQ, &q_full, (j * G + hl) * AD + c * 64,
                       p0, b);
+      IssuedFills k_fills, v_fills;
       // K tile i+1 is issued before V tile i: K stages free up as soon as their S MMA is done,
       // V stages only after P V, so the K loads run a tile further ahead
       auto load_k = [&](int i) -> bool {
@@ -251,6 +252,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         mbar_arrive_expect_tx(&k_full[st], KV_TILE_BYTES);
         tma_load_3d(kd, &tmK, &k_full[st], j * AD, t0, b);
         tma_load_3d(kd + KV_CHUNK, &tmK, &k_full[st], j * AD + 64, t0, b);
+        k_fills.note(st, (i / KV_STAGES) & 1);
         return true;
       };
       auto load_v = [&](int i) -> bool {
@@ -261,6 +263,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         mbar_arrive_expect_tx(&v_full[st], KV_TILE_BYTES);
         tma_load_3d(vd, &tmV, &v_full[st], j * AD, t0, b);
         tma_load_3d(vd + KV_CHUNK, &tmV, &v_full[st], j * AD + 64, t0, b);
+        v_fills.note(st, (i / KV_STAGES) & 1);
         return true;
       };
       if (n > 0 && load_k(0)) {
@@ -268,6 +271,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
           if (i + 1 < n && !load_k(i + 1)) break;
           if (!load_v(i)) break;
         }
+      }
+      if (*abort) {  // a wait expired: let the copies this thread issued land before the CTA exits
+        mbar_wait_drain(&q_full, 0);
+        k_fills.drain(k_full, KV_STAGES);
+        v_fills.drain(v_full, KV_STAGES);
       }
     }
   } else if (warp == 1) {
@@ -472,11 +480,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
 
   tc_fence_before();
   __syncthreads();
-  if (abort_flag) {
-    unsigned long long t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 1000000ull) {
-    }
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
+      IssuedFills fills;
       for (int t = blockIdx.x; t < total; t += gridDim.x) {
         int mt, nt;
         tm.map(t, mt, nt);
@@ -138,13 +139,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
           tma_load_2d(sa, &tmA, &full_bar[stage], kb * BK, mt * BM);
           tma_load_2d(sa + Cfg::A_BYTES, &tmB, &full_bar[stage], kb * BK, nt * BN);
+          fills.note(stage, phase);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-    producer_done:;
+    producer_done:
+      // a wait expired somewhere: let the copies this thread issued land before the CTA exits
+      if (*abort) fills.drain(full_bar, STAGES);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -338,10 +342,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i, q += p.N) hv[i] = i0 + i < nrows ? *q : 0.f;
             }
+            // rows at or beyond M (the ragged last row tile) touch no operand: their batch index
+            // would reach B and read past the caller's gate vector
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int bb = (row0 + i0 + i) / p.rows_per_batch;
-              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
+              if (i0 + i < nrows) {
+                const int bb = (row0 + i0 + i) / p.rows_per_batch;
+                hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
+              }
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i, hp += p.N)
@@ -356,12 +364,6 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
 
   __syncthreads();
-  if (abort_flag) {
-    // give TMA copies that may still be in flight time to land before the CTA exits
-    unsigned long long t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 1000000ull) {
-    }
-  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);

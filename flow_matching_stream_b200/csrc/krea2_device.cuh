@@ -88,6 +88,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits up to limit_ns for the phase of the given parity to complete, whatever the abort flag
+// says. The abort path uses it so that TMA copies already issued into shared memory land before
+// the CTA exits.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                unsigned long long limit_ns = WAIT_LIMIT_NS) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < limit_ns) {
+  }
+}
+
+// Stages a TMA producer has filled, with the phase parity of each one's last fill: on the abort
+// path the producer waits for exactly those fills. A completed fill stays observable under its
+// parity, because only the producer's next fill (which it no longer issues) advances the barrier.
+struct IssuedFills {
+  uint32_t mask = 0, parity = 0;
+  __device__ __forceinline__ void note(int stage, uint32_t ph) {
+    mask |= 1u << stage;
+    parity = (parity & ~(1u << stage)) | (ph << stage);
+  }
+  __device__ __forceinline__ void drain(uint64_t* full, int stages) const {
+    for (int s = 0; s < stages; ++s)
+      if ((mask >> s) & 1u) mbar_wait_drain(&full[s], (parity >> s) & 1u);
+  }
+};
+
 // ----------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

@@ -172,8 +172,9 @@ int krea2_gqa_attention(const Krea2Dims* dims, int B, int T, int N, int dtype,
  * 4369 tokens at the default 48/12 heads x 128) are rejected with KREA2_ERR_WORKSPACE before
  * anything runs. The call allocates and frees nothing. The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device current, so it should
- * come before any stream capture. All calls share the array and it keeps the last call's
- * contents (nothing in it needs to start at zero), so calls that overlap on the GPU race. */
+ * come before any stream capture. `stream` must belong to the current device (KREA2_ERR_ARG
+ * otherwise). All calls share the array and it keeps the last call's contents (nothing in it
+ * needs to start at zero), so calls that overlap on the GPU race. */
 #define KREA2_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int krea2_gqa_attention_noalloc(const Krea2Dims* dims, int B, int T, int N, int dtype,
                                 const void* qkvg, const float* q_norm_w, const float* k_norm_w,

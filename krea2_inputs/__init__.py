@@ -23,6 +23,8 @@ hidden_states (B, N, in_channels), position_ids (T + N, 3) with zero text rows a
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field, replace
 from typing import Dict, List, Optional, Sequence, Tuple
 
@@ -68,11 +70,17 @@ TINY = Dims(C=256, H=4, Hkv=1, D=64, F=512, axes=(16, 24, 24), n_layers=2, in_ch
 
 
 def to_bf16(x) -> np.ndarray:
-    """Round float32 values to the nearest bf16 value (ties to even); returns float32."""
+    """Round float32 values to the nearest bf16 value (ties to even); returns float32.
+
+    Adds 0x7FFF plus the lowest kept bit to the raw bits and clears the low 16 bits, in
+    wrapping 32-bit arithmetic (a new array; the input is left unchanged)."""
     x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
-    u = x.view(np.uint32).astype(np.uint64)
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return r.astype(np.uint32).view(np.float32).reshape(x.shape)
+    u = x.view(np.uint32)
+    r = (u >> np.uint32(16)) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32).reshape(x.shape)
 
 
 def bf16_bits(x) -> np.ndarray:
@@ -113,10 +121,11 @@ def block_weights(d: Dims, layer: int = 0, seed: int = SEED_WEIGHTS,
         "norm1_w": ((C,), 0.1), "norm2_w": ((C,), 0.1),
         "q_norm_w": ((D,), 0.1), "k_norm_w": ((D,), 0.1), "table": ((6, C), 0.1),
     }
-    out = {}
-    for i, name in enumerate(_BLOCK_TENSORS):
-        shape, std = shapes[name]
-        out[name] = _normal(seed, (layer, i), shape, std)
+    # every tensor has its own stream, so drawing them on threads (numpy releases the GIL while it
+    # fills an array) gives the same values as drawing them in turn
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        futs = {name: ex.submit(_normal, seed, (layer, i), *shapes[name]) for i, name in enumerate(_BLOCK_TENSORS)}
+        out = {name: futs[name].result() for name in _BLOCK_TENSORS}
     if zero_gates:
         out["table"][2] = 0.0
         out["table"][5] = 0.0

@@ -27,8 +27,10 @@ Readings where the pages are silent or garbled (the extraction of [ARCH] dropped
 ``+``, ``=`` operators of its block pseudo-code) are marked READING below.
 
 Parity status: every function here is pinned against closed forms, invariants, library
-routines or brute force: the block, backbone and their parts by ``tests/test_oracle_pins.py``,
-the sampler by ``tests/test_oracle_sampler.py``, text fusion by
+routines or brute force: the block, backbone and their parts (``img_in`` included) by
+``tests/test_oracle_pins.py``, the sampler pieces and the sampling loop (``sample_loop``
+against exact flows, ``sample``'s wiring of the two prompts) by
+``tests/test_oracle_sampler.py``, text fusion by
 ``tests/test_oracle_text_fusion.py``, and the block-causal pattern and cached step by
 ``tests/test_oracle_block_causal.py``. Agreement with the trained
 Krea 2 model itself is *unpinned*: no weights or reference outputs are available, and
@@ -382,27 +384,38 @@ def euler_step(x: np.ndarray, v: np.ndarray, sigma: float, sigma_next: float) ->
     return x + (sigma_next - sigma) * v
 
 
+def sample_loop(latents: np.ndarray, sigmas: Sequence[float], guidance: float,
+                velocity: Callable[[np.ndarray, float, int], np.ndarray], dtype=np.float64) -> np.ndarray:
+    """Sampling loop of [PIPE] __call__ for one image, with the model as a callable.
+
+    For i = 0 .. len(sigmas) - 2 the model is evaluated at the current latents and at timestep
+    sigmas[i] (t = sigma, [ARCH] §五): velocity(x, sigmas[i], 0) for the conditional prompt and,
+    when guidance > 0, velocity(x, sigmas[i], 1) for the unconditional one, as a separate call.
+    cfg_combine merges them and euler_step moves the latents from sigmas[i] to sigmas[i + 1].
+    Returns the final latents."""
+    x = latents.astype(dtype)
+    for i in range(len(sigmas) - 1):
+        vc = velocity(x, sigmas[i], 0)
+        vu = velocity(x, sigmas[i], 1) if guidance > 0 else None
+        x = euler_step(x, cfg_combine(vc, vu, guidance), sigmas[i], sigmas[i + 1])
+    return x
+
+
 def sample(latents: np.ndarray, text_cond: np.ndarray, text_uncond: Optional[np.ndarray],
            mask_cond: Optional[np.ndarray], mask_uncond: Optional[np.ndarray], pos: np.ndarray,
            sigmas: Sequence[float], guidance: float, mw: Dict[str, np.ndarray],
            block_w: Callable[[int], Dict[str, np.ndarray]], n_layers: int, H: int, Hkv: int, D: int,
            axes: Sequence[int], theta: float, eps: float, t_dim: int, dtype=np.float64) -> np.ndarray:
-    """Sampling loop of [PIPE] __call__ for one image: at each sigma the backbone predicts the
-    velocity for the conditional prompt (and, when guidance > 0, for the unconditional one, as
-    a separate forward), the two are combined with cfg_combine and euler_step moves the latents
-    to the next sigma. latents (N, in_ch); text_* (T, C); masks (T) or None. Returns (N, in_ch)."""
-    x = latents.astype(dtype)
-    for i in range(len(sigmas) - 1):
-        t = np.array([sigmas[i]], dtype=np.float64)
+    """sample_loop with the backbone as the model ([PIPE] __call__): branch 0 runs backbone_forward
+    on (text_cond, mask_cond), branch 1 on (text_uncond, mask_uncond), each as a batch of one at
+    timestep sigma. latents (N, in_ch); text_* (T, C); masks (T) or None. Returns (N, in_ch)."""
+    texts, masks = (text_cond, text_uncond), (mask_cond, mask_uncond)
 
-        def velocity(text, mask):
-            m = None if mask is None else mask[None]
-            return backbone_forward(x[None], text[None], pos, m, t, mw, block_w, n_layers, H, Hkv, D, axes,
-                                    theta, eps, t_dim, dtype)[0]
-        vc = velocity(text_cond, mask_cond)
-        vu = velocity(text_uncond, mask_uncond) if guidance > 0 else None
-        x = euler_step(x, cfg_combine(vc, vu, guidance), sigmas[i], sigmas[i + 1])
-    return x
+    def velocity(x, sigma, branch):
+        m = None if masks[branch] is None else masks[branch][None]
+        return backbone_forward(x[None], texts[branch][None], pos, m, np.array([sigma], dtype=np.float64), mw,
+                                block_w, n_layers, H, Hkv, D, axes, theta, eps, t_dim, dtype)[0]
+    return sample_loop(latents, sigmas, guidance, velocity, dtype)
 
 
 # ----------------------------------------------------------------------------- text fusion

@@ -486,6 +486,29 @@ def _backbone(d, B, T, gh, gw, lengths, layers=None, mw=None, zero_gates=False, 
                               d.theta, d.eps, d.t_dim, dtype)
 
 
+def test_img_in_against_torch_linear_with_bias():
+    # img_in = nn.Linear(in_channels, C, bias=True) ([ARCH] module list)
+    d = KI.TINY
+    mw = KI.model_weights(d)
+    x = KI.latents(d, 2, 24).astype(np.float64)
+    out = O.img_in(x, mw)
+    assert out.shape == (2, 24, d.C)
+    W, b = torch.from_numpy(mw["img_in_w"].astype(np.float64)), torch.from_numpy(mw["img_in_b"].astype(np.float64))
+    ref = Fn.linear(torch.from_numpy(x), W, b).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # negative control: the same check sees a dropped bias
+    assert np.max(np.abs(Fn.linear(torch.from_numpy(x), W).numpy() - out)) > 0.05
+
+
+def test_img_in_of_one_hot_latents_is_a_weight_column_plus_bias():
+    d = KI.TINY
+    mw = KI.model_weights(d)
+    out = O.img_in(np.eye(d.in_ch)[None], mw)[0]          # latent k = e_k
+    np.testing.assert_allclose(out, mw["img_in_w"].T.astype(np.float64) + mw["img_in_b"], rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(O.img_in(np.zeros((1, 3, d.in_ch)), mw)[0], np.tile(mw["img_in_b"], (3, 1)),
+                               rtol=0, atol=0)
+
+
 def test_quickstart_output_shape():
     g = _load("quickstart_shape.json")
     d = KI.with_dims(KI.tiny_block(), in_ch=g["in_channels"], n_layers=1).dims

@@ -10,8 +10,9 @@ CUDA events, an end-to-end pass through host buffers, and the CPU oracle on a bo
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
-Multi-GPU runs (torchrun, one rank per GPU) are replicas: each rank runs its own step with no
-data-path collective; time is the max over ranks.
+Multi-GPU runs are replicas: each rank runs its own step with no data-path collective; time is
+the max over ranks. Under torchrun WORLD_SIZE must equal --gpus; without a launcher, --gpus N > 1
+starts the N ranks itself (one process per GPU, rendezvous on 127.0.0.1).
 """
 from __future__ import annotations
 
@@ -397,10 +398,37 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample()
+    # last key: the figures the metric names, compact, so that the end of the line carries them
+    line["summary"] = summary(value / world, ms_step, pk, cfg_res, kernels, sweep)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def _r(x: float, sig: int = 4) -> float:
+    return float(f"{x:.{sig}g}")
+
+
+def summary(tflops_per_gpu: float, ms_step: float, pk: dict, cfg_res: dict, kernels: dict, sweep: list) -> dict:
+    """Compact figures for the end of the JSON line: the backbone step, the 1024^2 CFG block
+    (config 3) with its per-kernel fractions, attention's in-block share and the attention sweep."""
+    cfg_k = cfg_res["kernels"]
+    ker = {k: [_r(v["ms"]), _r(v["tflops"] if "tflops" in v else v["gbs"]),
+               _r(v["frac_sustained"] if "frac_sustained" in v else v["frac_hbm"], 3)]
+           for k, v in cfg_k.items() if k != "modulation"}
+    return {
+        "backbone_1024sq": {"ms_per_step": _r(ms_step), "tflops": _r(tflops_per_gpu),
+                            "frac_burst": _r(tflops_per_gpu / pk["bf16_tflops"], 3),
+                            "attention_share": _r(kernels["attention"]["share"], 3),
+                            "attention_frac_sustained": _r(kernels["attention"]["frac_sustained"], 3)},
+        "block_1024sq_cfg": {"ms": _r(cfg_res["ms_per_block"]), "tflops": _r(cfg_res["tflops"]),
+                             "frac_burst": _r(cfg_res["frac_burst"], 3),
+                             "frac_sustained": _r(cfg_res["frac_sustained"], 3),
+                             "kernels_ms_tflops_or_gbs_frac": ker},
+        "attention_sweep_grid_ms_tflops": [[s["grid"], _r(s["ms"]), _r(s["tflops"])] for s in sweep],
+        "peaks_source": pk["source"],
+    }
 
 
 def time_sampler(K2, torch, d, mw, dev) -> dict:
@@ -773,13 +801,50 @@ def main() -> None:
     if args.kernel_case:
         run_kernel_case(args.kernel_case, args.steps)
         return
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    launch = rank_layout(args.gpus, os.environ)
+    if launch == "spawn":
+        spawn_ranks(args)
+        return
+    rank, world, local_rank = launch
     if args.impl == "reference":
         run_reference(args, rank)
         return
     run_native(args, rank, world, local_rank)
+
+
+def rank_layout(gpus: int, env) -> object:
+    """(rank, world, local_rank) of this process, or "spawn" when --gpus N > 1 runs without a launcher.
+
+    Under torchrun WORLD_SIZE must equal --gpus: a mismatch would time a different number of
+    replicas than the line reports, so it stops the run."""
+    if gpus < 1:
+        raise SystemExit(f"--gpus must be >= 1, got {gpus}")
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != gpus:
+            raise SystemExit(f"WORLD_SIZE={world} from the launcher but --gpus {gpus}: they must agree")
+        return int(env.get("RANK", "0")), world, int(env.get("LOCAL_RANK", "0"))
+    return "spawn" if gpus > 1 else (0, 1, 0)
+
+
+def _spawned_rank(local_rank: int, args, port: int) -> None:
+    os.environ.update(RANK=str(local_rank), LOCAL_RANK=str(local_rank), WORLD_SIZE=str(args.gpus),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    if args.impl == "reference":
+        run_reference(args, local_rank)
+    else:
+        run_native(args, local_rank, args.gpus, local_rank)
+
+
+def spawn_ranks(args) -> None:
+    """One process per GPU on this node, as torchrun would start them (rendezvous on 127.0.0.1)."""
+    import socket
+
+    import torch.multiprocessing as mp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    mp.start_processes(_spawned_rank, args=(args, port), nprocs=args.gpus, start_method="spawn", join=True)
 
 
 if __name__ == "__main__":

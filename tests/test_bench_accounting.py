@@ -50,3 +50,31 @@ def test_both_arms_print_the_same_config():
     assert c["workload"] == wl.name and c["seq_len"] == 4608 and c["layers"] == 28
     assert abs(c["flops_per_step"] / 1e12 - 126.64) < 0.01
     assert c["parallelism"] == "single GPU" and bench.workload_config(wl, 8)["parallelism"] == "replicas"
+
+
+def test_rank_layout_guards_the_rank_count():
+    import pytest
+    assert bench.rank_layout(1, {}) == (0, 1, 0)
+    assert bench.rank_layout(4, {}) == "spawn"                      # no launcher: bench starts the ranks
+    env = {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"}
+    assert bench.rank_layout(2, env) == (1, 2, 1)
+    with pytest.raises(SystemExit):
+        bench.rank_layout(8, env)                                    # launcher and --gpus disagree
+    with pytest.raises(SystemExit):
+        bench.rank_layout(0, {})
+
+
+def test_summary_fits_the_tail_of_the_line():
+    # the driver keeps the last 1500 characters of the bench's output: the summary must fit in them
+    import json
+    pk = {"bf16_tflops": 1683.8, "bf16_tflops_sustained": 1391.3, "hbm_gbs": 6540.2, "source": "measured"}
+    names = ("modulation", "norm1", "qkv_proj", "attention", "out_proj_resid", "norm2", "gate_up_swiglu",
+             "down_proj_resid")
+    kern = {k: ({"ms": 0.123456, "tflops": 1234.5678, "frac_sustained": 0.87654, "share": 0.1}
+                if "proj" in k or k in ("attention", "gate_up_swiglu") else
+                {"ms": 0.0456789, "gbs": 4567.891, "frac_hbm": 0.698765, "share": 0.01}) for k in names}
+    cfg = {"ms_per_block": 7.2012345, "tflops": 1248.98765, "frac_burst": 0.7421234, "frac_sustained": 0.898765,
+           "kernels": kern}
+    sweep = [{"grid": g, "ms": 0.1234567, "tflops": 987.654321} for g in (32, 64, 96, 128)]
+    s = json.dumps({"summary": bench.summary(1119.123456, 113.123456, pk, cfg, kern, sweep)})
+    assert len(s) < 1300, len(s)

@@ -112,7 +112,7 @@ def test_attention_bf16_padded_keys_are_ignored(K2):
     np.testing.assert_array_equal(host(out2).reshape(B, S, d.HD), out)
 
 
-@pytest.mark.parametrize("grid", [32, 64, 128])
+@pytest.mark.parametrize("grid", [32, 64, 96, 128])
 def test_attention_sweep_sampled_rows(K2, grid):
     # the attention-only sweep shapes (512 text tokens, random valid length), rows sampled
     wl = KI.attn_sweep(grid)
@@ -122,6 +122,22 @@ def test_attention_sweep_sampled_rows(K2, grid):
     rows = sample_rows(wl.T, wl.S)
     ref = oracle_attention(d, x, w, pos, wl.B, wl.T, wl.N, mask, rows=rows, dtype=np.float32)
     assert rel_err(out[:, rows], ref) < TOL_BF16
+
+
+@pytest.mark.parametrize("T,length", [(512, 512), (509, 301)])
+def test_attention_full_size_whole_cta_tiles(K2, T, length):
+    # Full heads at the 1024^2 sequence length: every row (all 48 heads) of the query tiles around the
+    # text/image boundary and of the last tiles of the sequence. T = 509 makes S = 4605 ragged: the
+    # last tile is partial and a tile straddles the boundary under 32- and 64-position tilings alike.
+    d = KI.FULL
+    B, gh, gw = 1, 64, 64
+    S = T + gh * gw
+    mask = KI.mask_from_lengths(T, [length])
+    x, w, pos, out = run_attention(K2, d, B, T, gh, gw, mask, torch.bfloat16, key=3)
+    lo = (T // 64) * 64
+    rows = sorted(set(range(lo - 64, min(lo + 128, S))) | set(range((S // 64) * 64 - 64, S)))
+    ref = oracle_attention(d, x, w, pos, B, T, gh * gw, mask, rows=rows, dtype=np.float32)
+    assert rel_err(out[:, rows], ref, f"S={S}, {len(rows)} rows") < TOL_BF16
 
 
 @pytest.mark.parametrize("H,Hkv", [(8, 8), (8, 4), (20, 20)])

@@ -55,6 +55,35 @@ def test_backbone_full_width_two_layers_bf16(K2):
     assert rel_err(vel, ref) < TOL_BF16
 
 
+def test_backbone_28_layers_full_width_live_gates(K2):
+    # All 28 full-width blocks, each with its own seeded weights and live gates, on a short sequence
+    # (2 batch rows of 64 text tokens, the second padded to 20 valid, plus an 8x8 image) so that the
+    # fp32 oracle finishes in seconds. Tolerance: the per-block bf16 bound, unchanged for the stack.
+    d = KI.FULL
+    B, T, gh, gw, lengths = 2, 64, 8, 8, [64, 20]
+    N = gh * gw
+    mw_h = KI.model_weights(d)
+    blocks = []
+
+    def block_w(i):  # the oracle draws each block once; the same weights go to the device
+        w = KI.block_weights(d, i)
+        blocks.append(K2.BlockWeights(w, torch.bfloat16, "cuda"))
+        return w
+    hidden, text = KI.latents(d, B, N), KI.text_states(d, B, T)
+    pos, mask, t = KI.position_ids(T, gh, gw), KI.mask_from_lengths(T, lengths), KI.timesteps(B)
+    ref = O.backbone_forward(hidden, text, pos, mask, t, mw_h, block_w, d.n_layers, d.H, d.Hkv, d.D, d.axes,
+                             d.theta, d.eps, d.t_dim, np.float32)
+    assert len(blocks) == d.n_layers == 28
+    vel, _ = run_backbone(K2, d, B, T, gh, gw, lengths, torch.bfloat16, mw_h=mw_h, blocks=blocks)
+    assert rel_err(vel, ref, "28 layers, live gates") < TOL_BF16
+    # the gates are live: the stack moves the velocity far from that of identity blocks
+    _, e = O.time_path(t, mw_h, d.t_dim, np.float32)
+    identity = O.final_layer(O.img_in(hidden, mw_h, np.float32), e, mw_h, d.eps, np.float32)
+    assert rel_err(identity, ref, "identity blocks vs live") > 0.1
+    del blocks
+    torch.cuda.empty_cache()
+
+
 def test_backbone_quickstart_shape(K2):
     # 16 text tokens + 8x8 latent grid -> velocity (1, 64, 64) (quick-start example of the pages)
     d = KI.with_dims(KI.backbone_1024(), n_layers=1).dims

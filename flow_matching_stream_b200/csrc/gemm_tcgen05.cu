@@ -214,9 +214,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const int nrows = min(32, p.M - row0);
       uint32_t* xpk = reinterpret_cast<uint32_t*>(base + STAGES * Cfg::STAGE_BYTES) + (warp - 2) * (32 * 33);
       if constexpr (EPI == EPI_STORE) {
-        __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row0 * p.N + (size_t)nt * BN;
+        const int ld = p.out_ld ? p.out_ld : p.N;
+        const int n_store = p.n_store ? p.n_store : p.N;
+        __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row0 * ld + (size_t)nt * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 64; ++c) {
+          if (nt * BN + c * 64 >= n_store) break;  // warp-uniform: padding columns of W are not stored
           float v[64];
           tmem_ld64(tbase + c * 64, v);
           if (p.bias) {
@@ -233,7 +236,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-          store_bf16_rows(xpk, pk, out0 + c * 64, p.N, nrows, lane);
+          store_bf16_rows(xpk, pk, out0 + c * 64, ld, nrows, lane);
+        }
+      } else if constexpr (EPI == EPI_BIAS_ROWMAP) {
+        // fp32 out[map(row), col] = acc + bias[col], rows transposed through shared memory like the
+        // residual epilogue below; lane i holds the destination row of tile row row0 + i
+        float* xp = reinterpret_cast<float*>(xpk);
+        const int rr = min(row0 + lane, p.M - 1);
+        const long long my_dst = (long long)(rr / p.map_N) * p.map_S + p.map_T + rr % p.map_N;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = v[e];
+          __syncwarp();
+          const int col = nt * BN + c * 32 + lane;
+          const float bv = p.bias ? __ldg(p.bias + col) : 0.f;
+          float* out = reinterpret_cast<float*>(p.out) + col;
+#pragma unroll 8
+          for (int i = 0; i < 32; ++i) {
+            const long long dst = __shfl_sync(0xffffffffu, my_dst, i);
+            if (i < nrows) out[dst * p.N] = xp[i * 33 + lane] + bv;
+          }
+          __syncwarp();
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
         // interleaved 64-row groups: columns [128g, 128g+64) gate, [128g+64, 128g+128) up
@@ -324,7 +350,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // L1 wavefront each, in the SRAM that also feeds the tensor core), so the warp
         // transposes its 32x32 block through a padded shared tile and then walks the rows: each
         // access is one 128-byte line, and 16 rows of loads are in flight before any store.
+        // Lane i knows the batch row of tile row row0 + i (clamped to M - 1, so that rows of the
+        // ragged last tile read an in-bounds gate; their results are never stored).
         float* xp = reinterpret_cast<float*>(xpk);
+        const int my_b = min(row0 + lane, p.M - 1) / p.rows_per_batch;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
@@ -337,23 +366,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           for (int i0 = 0; i0 < 32; i0 += 16) {
             float* hp = reinterpret_cast<float*>(p.out) + (size_t)(row0 + i0) * p.N + col;
             float hv[16];
-            {
-              const float* q = hp;
 #pragma unroll
-              for (int i = 0; i < 16; ++i, q += p.N) hv[i] = i0 + i < nrows ? *q : 0.f;
-            }
-            // rows at or beyond M (the ragged last row tile) touch no operand: their batch index
-            // would reach B and read past the caller's gate vector
+            for (int i = 0; i < 16; ++i) hv[i] = i0 + i < nrows ? hp[(size_t)i * p.N] : 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              if (i0 + i < nrows) {
-                const int bb = (row0 + i0 + i) / p.rows_per_batch;
-                hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
-              }
+              const int bb = __shfl_sync(0xffffffffu, my_b, i0 + i);
+              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i, hp += p.N)
-              if (i0 + i < nrows) *hp = hv[i];
+            for (int i = 0; i < 16; ++i)
+              if (i0 + i < nrows) hp[(size_t)i * p.N] = hv[i];
           }
           __syncwarp();
         }
@@ -443,7 +465,7 @@ int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStrea
   CUtensorMap ta, tb;
   int rc = make_tmap_bf16_2d(&ta, A, p0.K, p0.M, p0.K, BK, BM);
   if (rc) return rc;
-  rc = make_tmap_bf16_2d(&tb, W, p0.K, p0.N, p0.K, BK, BN);
+  rc = make_tmap_bf16_2d(&tb, W, p0.K, p0.w_rows ? p0.w_rows : p0.N, p0.K, BK, BN);
   if (rc) return rc;
   GemmParams p = p0;
   p.tiles_m = (p.M + BM - 1) / BM;
@@ -488,6 +510,7 @@ int gemm_bf16(int epi, const GemmParams& p, const void* A, const void* W, cudaSt
       case EPI_STORE: return launch_gemm_bn<256, EPI_STORE>(p, A, W, stream);
       case EPI_SWIGLU: return launch_gemm_bn<256, EPI_SWIGLU>(p, A, W, stream);
       case EPI_QKV: return launch_gemm_bn<256, EPI_QKV>(p, A, W, stream);
+      case EPI_BIAS_ROWMAP: return launch_gemm_bn<256, EPI_BIAS_ROWMAP>(p, A, W, stream);
       default: return launch_gemm_bn<256, EPI_RESID>(p, A, W, stream);
     }
   }
@@ -495,6 +518,7 @@ int gemm_bf16(int epi, const GemmParams& p, const void* A, const void* W, cudaSt
     case EPI_STORE: return launch_gemm_bn<128, EPI_STORE>(p, A, W, stream);
     case EPI_SWIGLU: return launch_gemm_bn<128, EPI_SWIGLU>(p, A, W, stream);
     case EPI_QKV: return launch_gemm_bn<128, EPI_QKV>(p, A, W, stream);
+    case EPI_BIAS_ROWMAP: return launch_gemm_bn<128, EPI_BIAS_ROWMAP>(p, A, W, stream);
     default: return launch_gemm_bn<128, EPI_RESID>(p, A, W, stream);
   }
 }

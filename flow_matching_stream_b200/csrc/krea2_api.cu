@@ -179,6 +179,43 @@ int check_model_weights(const Krea2ModelWeights* w, int n_layers) {
   return KREA2_OK;
 }
 
+// Final layer ([ARCH] §四.6). With a bf16 scratch of B*N*C (final_layer_tc_scratch) the modulated
+// norm of the image rows goes to the scratch and the projection runs on the tensor cores (W rows
+// beyond in_ch read as zeros, only in_ch columns are stored); otherwise one fused SIMT kernel.
+int final_layer_impl(const Krea2Dims* d, int B, int T, int N, bool bf, const float* h, const float* e,
+                     const Krea2ModelWeights* w, void* velocity, void* scratch, cudaStream_t s) {
+  if (!scratch || !final_layer_tc_scratch(d, B, N, bf)) return launch_final_layer(d, B, T, N, bf, h, e, w, velocity, s);
+  ModNormArgs a{};
+  a.h = h; a.w = w->final_norm_w;
+  a.sc = e; a.sh = e; a.mod_stride = d->C;  // (scale, shift) = final_table + e ([ARCH] §四.6, reading c16)
+  a.sc_tab = w->final_table; a.sh_tab = w->final_table + d->C;
+  a.B = B; a.rows = N; a.S_in = T + N; a.row0 = T; a.C = d->C; a.eps = d->eps;
+  a.out = scratch; a.out_bf16 = true;
+  int rc = launch_mod_rmsnorm_rows(a, s);
+  if (rc) return rc;
+  GemmParams gp{};
+  gp.M = B * N; gp.N = (d->in_ch + 127) / 128 * 128; gp.K = d->C; gp.out = velocity; gp.bias = w->final_b;
+  gp.out_ld = d->in_ch; gp.n_store = d->in_ch; gp.w_rows = d->in_ch;
+  return gemm_bf16(EPI_STORE, gp, scratch, w->final_w, s);
+}
+
+// img_in = Linear(in_ch, C, bias=True) on the packed latents, written to the image rows of the
+// residual (after the T text rows of each batch row) ([ARCH] §四 module list and data flow).
+int img_in_impl(const Krea2Dims* d, int B, int T, int N, bool bf, const void* hidden, const Krea2ModelWeights* w,
+                float* h, cudaStream_t s) {
+  const int S = T + N, C = d->C;
+  if (bf && d->in_ch % 64 == 0) {
+    GemmParams gp{};
+    gp.M = B * N; gp.N = C; gp.K = d->in_ch; gp.out = h; gp.bias = w->img_in_b;
+    gp.map_N = N; gp.map_T = T; gp.map_S = S;
+    return gemm_bf16(EPI_BIAS_ROWMAP, gp, hidden, w->img_in_w, s);
+  }
+  SimtGemmParams ip{};
+  ip.M = B * N; ip.N = C; ip.K = d->in_ch; ip.out = h; ip.bias = w->img_in_b;
+  ip.map_N = N; ip.map_T = T; ip.map_S = S;
+  return gemm_simt(SEPI_BIAS_ROWMAP, ip, hidden, bf, w->img_in_w, bf, s);
+}
+
 // The block's launch sequence ([ARCH] §四.2) on an already validated configuration.
 int block_impl(const Krea2Dims* d, int B, int T, int N, int dtype, float* h, const float* temb,
                const Krea2BlockWeights* w, const float* cs, const float* sn, const uint8_t* mask, uint8_t* ws,
@@ -267,6 +304,12 @@ int krea2_check_device_error(void* stream) {
 int krea2_selftest_wait_timeout(int limit_ms, int* waited, void* stream) {
   if (limit_ms < 1 || limit_ms > 5000 || !waited) return set_error(KREA2_ERR_ARG, "limit_ms must be 1..5000, waited non-NULL");
   return launch_wait_timeout_selftest((unsigned long long)limit_ms * 1000000ull, waited, as_stream(stream));
+}
+
+int krea2_selftest_exp2_poly(const float* x, float* y, long long n, void* stream) {
+  if (!x || !y || n < 0 || (n & 1)) return set_error(KREA2_ERR_ARG, "need x, y non-NULL and an even n >= 0");
+  if (n == 0) return KREA2_OK;
+  return launch_exp2_poly_selftest(x, y, n, as_stream(stream));
 }
 
 size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype) {
@@ -444,13 +487,23 @@ int krea2_time_embed(const Krea2Dims* dims, int B, int dtype, const float* times
   return launch_time_embed(dims, B, dtype == KREA2_BF16, timestep, w, temb_out, e_out, scratch, as_stream(stream));
 }
 
+size_t krea2_final_layer_workspace_size(const Krea2Dims* dims, int B, int N, int dtype) {
+  if (check_dims(dims, dtype) || check_model_dims(dims) || check_shape(B, 0, N)) return 0;
+  return final_layer_tc_scratch(dims, B, N, dtype == KREA2_BF16);
+}
+
 int krea2_final_layer(const Krea2Dims* dims, int B, int T, int N, int dtype, const float* h, const float* e,
-                      const Krea2ModelWeights* w, void* velocity, void* stream) {
+                      const Krea2ModelWeights* w, void* velocity, void* workspace, size_t ws_bytes, void* stream) {
   int rc = check_dims(dims, dtype);
   if (rc || (rc = check_model_dims(dims)) || (rc = check_shape(B, T, N))) return rc;
   if (!h || !e || !w || !w->final_norm_w || !w->final_table || !w->final_w || !w->final_b || !velocity)
     return set_error(KREA2_ERR_ARG, "NULL pointer");
-  return launch_final_layer(dims, B, T, N, dtype == KREA2_BF16, h, e, w, velocity, as_stream(stream));
+  const size_t need = final_layer_tc_scratch(dims, B, N, dtype == KREA2_BF16);
+  if (need && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)))
+    return set_error(KREA2_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (ws_bytes < need) return set_error(KREA2_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return final_layer_impl(dims, B, T, N, dtype == KREA2_BF16, h, e, w, velocity, need ? workspace : nullptr,
+                          as_stream(stream));
 }
 
 int krea2_block_forward(const Krea2Dims* dims, int B, int T, int N, int dtype, float* h, const float* temb,
@@ -733,14 +786,12 @@ int krea2_backbone_forward(const Krea2Dims* dims, int B, int T, int N, int dtype
     return rc;
   if ((rc = launch_time_embed(dims, B, bf, timestep, w, temb, e, reinterpret_cast<float*>(ws + L.tscr), s))) return rc;
   if ((rc = launch_copy_text_rows(text_states, bf, B, T, S, C, h, s))) return rc;
-  SimtGemmParams ip{};
-  ip.M = B * N; ip.N = C; ip.K = dims->in_ch; ip.out = h; ip.bias = w->img_in_b;
-  ip.map_N = N; ip.map_T = T; ip.map_S = S;
-  if ((rc = gemm_simt(SEPI_BIAS_ROWMAP, ip, hidden_states, bf, w->img_in_w, bf, s))) return rc;
+  if ((rc = img_in_impl(dims, B, T, N, bf, hidden_states, w, h, s))) return rc;
   const uint8_t* mask = T > 0 ? text_mask : nullptr;
   for (int l = 0; l < dims->n_layers; ++l)
     if ((rc = block_impl(dims, B, T, N, dtype, h, temb, &w->blocks[l], cs, sn, mask, ws, L, s))) return rc;
-  return launch_final_layer(dims, B, T, N, bf, h, e, w, velocity, s);
+  // the block activations are dead now: their bf16 xn buffer (B*S*C) holds the final norm's output
+  return final_layer_impl(dims, B, T, N, bf, h, e, w, velocity, ws + L.xn, s);
 }
 
 }  // extern "C"

@@ -9,7 +9,10 @@
 
 namespace krea2 {
 
-enum { EPI_STORE = KREA2_EPI_STORE, EPI_SWIGLU = KREA2_EPI_SWIGLU, EPI_RESID = KREA2_EPI_RESID, EPI_QKV = 3 };
+// EPI_BIAS_ROWMAP: fp32 out[map(row), col] = acc + bias[col], map(r) = (r / map_N) * map_S + map_T + r % map_N
+// (img_in writing the image rows of the residual after the text rows).
+enum { EPI_STORE = KREA2_EPI_STORE, EPI_SWIGLU = KREA2_EPI_SWIGLU, EPI_RESID = KREA2_EPI_RESID, EPI_QKV = 3,
+       EPI_BIAS_ROWMAP = 4 };
 
 // Records a message for krea2_last_error_string() and returns `code`.
 int set_error(int code, const char* fmt, ...);
@@ -42,6 +45,10 @@ struct GemmParams {
   const float* sin;
   int HD, KVD;
   float eps;
+  int out_ld;               // STORE: row stride of out in elements (0: N)
+  int n_store;              // STORE: columns stored, a multiple of 64 (0: N)
+  int w_rows;               // rows of W present (0: N); rows beyond read as zeros
+  int map_N, map_T, map_S;  // BIAS_ROWMAP row map
   int tiles_m, tiles_n;     // filled by the launcher
   int group_m;              // row tiles per raster group (filled by the launcher)
 };
@@ -73,10 +80,28 @@ int launch_modulation(const float* temb, const float* table, int B, int C, float
 // (then temb already holds temb+table).
 int launch_mod_rmsnorm(const float* h, const float* w, const float* temb, const float* table, int chunk, int B, int S,
                        int C, float eps, void* out, bool out_bf16, cudaStream_t stream);
+// General form: output row r (of B * rows) reads h row (r / rows) * S_in + row0 + r % rows;
+// scale = sc[b * mod_stride + c] (+ sc_tab[c]), shift = sh[b * mod_stride + c] (+ sh_tab[c]).
+struct ModNormArgs {
+  const float* h;
+  const float* w;
+  const float* sc;
+  const float* sh;
+  long long mod_stride;
+  const float* sc_tab;  // nullable
+  const float* sh_tab;  // nullable
+  int B, rows, S_in, row0, C;
+  float eps;
+  void* out;
+  bool out_bf16;
+};
+int launch_mod_rmsnorm_rows(const ModNormArgs& a, cudaStream_t stream);
 int launch_time_embed(const Krea2Dims* d, int B, bool w_bf16, const float* t, const Krea2ModelWeights* w,
                       float* temb, float* e, float* scratch, cudaStream_t stream);
 int launch_final_layer(const Krea2Dims* d, int B, int T, int N, bool bf16, const float* h, const float* e,
                        const Krea2ModelWeights* w, void* velocity, cudaStream_t stream);
+// Bytes of bf16 scratch the tensor-core final layer needs (0 when it does not apply).
+size_t final_layer_tc_scratch(const Krea2Dims* d, int B, int N, bool bf16);
 int launch_euler_cfg(bool bf16, long long n, float* x, const void* vc, const void* vu, float g, float sigma,
                      float sigma_next, void* xm, int copies, float* t_out, cudaStream_t stream);
 int launch_unit_modulation(int B, int C, float* mod, cudaStream_t stream);
@@ -117,6 +142,7 @@ struct AttnTcArgs {
 };
 bool attention_tc_supported(int D, int H, int Hkv);
 int launch_wait_timeout_selftest(unsigned long long limit_ns, int* waited, cudaStream_t stream);
+int launch_exp2_poly_selftest(const float* x, float* y, long long n, cudaStream_t stream);
 int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream);
 // raw k and v of n tokens -> rows [row0, row0 + n) of every batch row of a key/value cache
 // (k RMS-normalised and rotated, v copied; bf16, (B, capacity, Hkv*128))

@@ -100,16 +100,17 @@ __global__ void from_f32_kernel(const float* __restrict__ in, long n, void* __re
 }
 
 // ----------------------------------------------------------------------------- modulated RMSNorm
-// One CTA per row; C % 4 == 0; 256 threads, float4 loads of the fp32 residual.
+// One CTA per output row; C % 4 == 0; 256 threads, float4 loads of the fp32 residual.
+// Output row r reads residual row (r / rows) * S_in + row0 + r % rows (the identity for the block
+// norms; the image rows for the final layer) and batch b = r / rows picks the modulation vectors.
 template <bool OUT_BF16>
-__global__ void __launch_bounds__(256) mod_rmsnorm_kernel(const float* __restrict__ h, const float* __restrict__ w,
-                                                          const float* __restrict__ temb,
-                                                          const float* __restrict__ table, int chunk, int S, int C,
-                                                          float eps, void* __restrict__ out) {
+__global__ void __launch_bounds__(256) mod_rmsnorm_kernel(ModNormArgs a) {
   const long row = blockIdx.x;
-  const int b = (int)(row / S);
+  const int C = a.C;
+  const int b = (int)(row / a.rows);
+  const long in_row = (long)b * a.S_in + a.row0 + row % a.rows;
   const int C4 = C >> 2;
-  const float4* x4 = reinterpret_cast<const float4*>(h + row * C);
+  const float4* x4 = reinterpret_cast<const float4*>(a.h + in_row * C);
   constexpr int MAXV = 8;  // up to C = 8192
   float4 xv[MAXV];
   float ss = 0.f;
@@ -128,24 +129,22 @@ __global__ void __launch_bounds__(256) mod_rmsnorm_kernel(const float* __restric
   float tot = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) tot += red[i];
-  const float r = rsqrtf(tot / (float)C + eps);
-  const float* sc_t = temb + (long)b * 6 * C + (long)chunk * C;
-  const float* sh_t = sc_t + C;
-  const float* sc_b = table ? table + (long)chunk * C : nullptr;
-  const float* sh_b = table ? sc_b + C : nullptr;
+  const float r = rsqrtf(tot / (float)C + a.eps);
+  const float* sc_t = a.sc + (long)b * a.mod_stride;
+  const float* sh_t = a.sh + (long)b * a.mod_stride;
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int c4 = threadIdx.x + i * 256;
     if (c4 < C4) {
       const int c = c4 * 4;
-      float4 ww = *reinterpret_cast<const float4*>(w + c);
-      float4 sc = *reinterpret_cast<const float4*>(sc_t + c);
-      float4 sh = *reinterpret_cast<const float4*>(sh_t + c);
-      if (table) {
-        const float4 a = *reinterpret_cast<const float4*>(sc_b + c);
-        const float4 bb = *reinterpret_cast<const float4*>(sh_b + c);
-        sc.x += a.x; sc.y += a.y; sc.z += a.z; sc.w += a.w;
-        sh.x += bb.x; sh.y += bb.y; sh.z += bb.z; sh.w += bb.w;
+      float4 ww = __ldg(reinterpret_cast<const float4*>(a.w + c));
+      float4 sc = __ldg(reinterpret_cast<const float4*>(sc_t + c));
+      float4 sh = __ldg(reinterpret_cast<const float4*>(sh_t + c));
+      if (a.sc_tab) {
+        const float4 t0 = __ldg(reinterpret_cast<const float4*>(a.sc_tab + c));
+        const float4 t1 = __ldg(reinterpret_cast<const float4*>(a.sh_tab + c));
+        sc.x += t0.x; sc.y += t0.y; sc.z += t0.z; sc.w += t0.w;
+        sh.x += t1.x; sh.y += t1.y; sh.z += t1.z; sh.w += t1.w;
       }
       float y0 = (1.f + sc.x) * (xv[i].x * r * (1.f + ww.x)) + sh.x;
       float y1 = (1.f + sc.y) * (xv[i].y * r * (1.f + ww.y)) + sh.y;
@@ -155,9 +154,9 @@ __global__ void __launch_bounds__(256) mod_rmsnorm_kernel(const float* __restric
         uint2 o;
         o.x = pack_bf16x2(y0, y1);
         o.y = pack_bf16x2(y2, y3);
-        reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + row * C)[c4] = o;
+        reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + row * C)[c4] = o;
       } else {
-        reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + row * C)[c4] = make_float4(y0, y1, y2, y3);
+        reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + row * C)[c4] = make_float4(y0, y1, y2, y3);
       }
     }
   }
@@ -183,6 +182,8 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
 }
 
 // out[b, n] = act(sum_k x[b, k] W[n, k] + bias[n]); one warp per output feature, all batch rows.
+// The K loop is unrolled by 4 so that each lane keeps four 16-byte weight loads in flight: the
+// weights stream from HBM once per forward and this kernel is bound by that stream.
 template <bool W_BF16, bool GELU>
 __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __restrict__ x, const void* __restrict__ W,
                                                              const float* __restrict__ bias, int B, int N, int K,
@@ -195,6 +196,7 @@ __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __rest
     float acc[MAXB];
 #pragma unroll
     for (int b = 0; b < MAXB; ++b) acc[b] = 0.f;
+#pragma unroll 4
     for (int k = lane * 8; k < K; k += 256) {
       float wv[8];
       if (W_BF16) {
@@ -599,15 +601,23 @@ int launch_to_dtype(const float* in, long n, void* out, bool out_bf16, cudaStrea
   return check_launch("to_dtype");
 }
 
+int launch_mod_rmsnorm_rows(const ModNormArgs& a, cudaStream_t stream) {
+  const long rows = (long)a.B * a.rows;
+  if (rows == 0) return KREA2_OK;
+  if (a.out_bf16) mod_rmsnorm_kernel<true><<<(unsigned)rows, 256, 0, stream>>>(a);
+  else mod_rmsnorm_kernel<false><<<(unsigned)rows, 256, 0, stream>>>(a);
+  return check_launch("mod_rmsnorm");
+}
+
 int launch_mod_rmsnorm(const float* h, const float* w, const float* temb, const float* table, int chunk, int B, int S,
                        int C, float eps, void* out, bool out_bf16, cudaStream_t stream) {
-  const long rows = (long)B * S;
-  if (rows == 0) return KREA2_OK;
-  if (out_bf16)
-    mod_rmsnorm_kernel<true><<<(unsigned)rows, 256, 0, stream>>>(h, w, temb, table, chunk, S, C, eps, out);
-  else
-    mod_rmsnorm_kernel<false><<<(unsigned)rows, 256, 0, stream>>>(h, w, temb, table, chunk, S, C, eps, out);
-  return check_launch("mod_rmsnorm");
+  ModNormArgs a{};
+  a.h = h; a.w = w;
+  a.sc = temb + (long)chunk * C; a.sh = temb + (long)(chunk + 1) * C; a.mod_stride = 6LL * C;
+  a.sc_tab = table ? table + (long)chunk * C : nullptr;
+  a.sh_tab = table ? table + (long)(chunk + 1) * C : nullptr;
+  a.B = B; a.rows = S; a.S_in = S; a.row0 = 0; a.C = C; a.eps = eps; a.out = out; a.out_bf16 = out_bf16;
+  return launch_mod_rmsnorm_rows(a, stream);
 }
 
 int launch_time_embed(const Krea2Dims* d, int B, bool w_bf16, const float* t, const Krea2ModelWeights* w,
@@ -631,6 +641,11 @@ int launch_time_embed(const Krea2Dims* d, int B, bool w_bf16, const float* t, co
   if ((rc = lin(e, w->t1_w, w->t1_b, C, td, scratch, true))) return rc;
   if ((rc = lin(scratch, w->t2_w, w->t2_b, C, C, e, true))) return rc;
   return lin(e, w->mod_w, w->mod_b, 6 * C, C, temb, false);
+}
+
+size_t final_layer_tc_scratch(const Krea2Dims* d, int B, int N, bool bf16) {
+  if (!bf16 || d->in_ch % 64) return 0;
+  return (size_t)B * N * d->C * 2;
 }
 
 int launch_final_layer(const Krea2Dims* d, int B, int T, int N, bool bf16, const float* h, const float* e,

@@ -20,7 +20,7 @@ from ._lib import KREA2_BF16, KREA2_F32, KREA2_EPI_RESID, KREA2_EPI_STORE, KREA2
 __all__ = [
     "Krea2Error", "lib", "dims_struct", "dtype_code", "workspace_size", "attention_workspace_size",
     "rope_tables", "gqa_attention", "gqa_attention_noalloc", "block_causal_key_end", "gqa_attention_block_causal",
-    "kv_cache_append", "kv_cache_attention_workspace_size", "gqa_attention_kv_cache", "modulated_rmsnorm", "linear", "time_embed", "final_layer",
+    "kv_cache_append", "kv_cache_attention_workspace_size", "gqa_attention_kv_cache", "modulated_rmsnorm", "linear", "time_embed", "final_layer_workspace_size", "final_layer",
     "text_dims_struct", "TextWeights", "text_fusion_workspace_size", "text_fusion",
     "shift_mu", "sigma_schedule", "euler_cfg_step", "sample_workspace_size", "sample",
     "block_forward", "block_forward_traced", "BLOCK_STEPS", "launch_count", "backbone_forward", "check_device_error", "BlockWeights", "ModelWeights",
@@ -206,10 +206,15 @@ def time_embed(dims, timestep: torch.Tensor, mw: "ModelWeights", temb_out: torch
                                   ctypes.byref(mw.struct), _p(temb_out), _p(e_out), _p(scratch), _s(stream)))
 
 
+def final_layer_workspace_size(dims, B: int, N: int, dtype: torch.dtype) -> int:
+    return int(lib().krea2_final_layer_workspace_size(ctypes.byref(dims_struct(dims)), B, N, dtype_code(dtype)))
+
+
 def final_layer(dims, B: int, T: int, N: int, h: torch.Tensor, e: torch.Tensor, mw: "ModelWeights",
-                velocity: torch.Tensor, stream=None) -> None:
+                velocity: torch.Tensor, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().krea2_final_layer(ctypes.byref(dims_struct(dims)), B, T, N, mw.dtype_code, _p(h), _p(e),
-                                   ctypes.byref(mw.struct), _p(velocity), _s(stream)))
+                                   ctypes.byref(mw.struct), _p(velocity), _p(workspace), ws, _s(stream)))
 
 
 def block_forward(dims, B: int, T: int, N: int, h: torch.Tensor, temb: torch.Tensor, bw: "BlockWeights",

@@ -128,6 +128,13 @@ int krea2_check_device_error(void* stream);
  * KREA2_ERR_TIMEOUT and clears the error word. The context stays usable. */
 int krea2_selftest_wait_timeout(int limit_ms, int* waited, void* stream);
 
+/* Numerics self-test of the attention kernel's exp2 on the FMA pipe (no counterpart in the pages:
+ * the softmax of [ARCH] §四.3 needs exp, and the tensor-core attention evaluates some of its
+ * exponentials with a cubic instead of the MUFU). x, y: n fp32 DEVICE values, n even; writes
+ * y[i] ~ 2^x[i] for x[i] in [-125, 8.5] with at most 7.5e-5 relative error (the fit's bound);
+ * below -125 the result is about 2^-125. KREA2_ERR_ARG for odd n or NULL pointers. */
+int krea2_selftest_exp2_poly(const float* x, float* y, long long n, void* stream);
+
 /* Bytes of device workspace that krea2_block_forward / krea2_backbone_forward need for
  * these shapes (0 on invalid arguments). The workspace must be 256-byte aligned. */
 size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype);
@@ -276,10 +283,14 @@ int krea2_time_embed(const Krea2Dims* dims, int B, int dtype, const float* times
 /* Final layer on image rows ([ARCH] §四.6): (scale, shift) = final_table + e;
  * y = (1 + scale) * rms(x) * (1 + final_norm_w) + shift; velocity = y · final_wᵀ + final_b.
  * h (B*S, C) fp32 full sequence (text rows are skipped, [ARCH] §二); e (B, C) fp32;
- * velocity (B, N, in_ch) in `dtype` (in_ch <= 64). Reads w->final_*. One fused kernel. */
+ * velocity (B, N, in_ch) in `dtype` (in_ch <= 64). Reads w->final_*.
+ * workspace: krea2_final_layer_workspace_size bytes, 256-byte aligned (NULL allowed when that is
+ * 0). bf16 with in_ch % 64 == 0: the norm writes y (bf16) there and the projection runs on the
+ * tensor cores; otherwise one fused SIMT kernel (no workspace). */
+size_t krea2_final_layer_workspace_size(const Krea2Dims* dims, int B, int N, int dtype);
 int krea2_final_layer(const Krea2Dims* dims, int B, int T, int N, int dtype,
                       const float* h, const float* e, const Krea2ModelWeights* w,
-                      void* velocity, void* stream);
+                      void* velocity, void* workspace, size_t ws_bytes, void* stream);
 
 /* One Krea2TransformerBlock forward ([ARCH] §四.2), in place on the fp32 residual:
  *   mod = temb + table;  xn = (1+prescale)*norm1(h) + preshift;

@@ -56,7 +56,6 @@ SIGNATURES = {
     "krea2_check_device_error": (c_int, [V]),
     "krea2_workspace_size": (c_size_t, [_PD, c_int, c_int, c_int, c_int]),
     "krea2_selftest_wait_timeout": (c_int, [c_int, V, V]),
-    "krea2_selftest_exp2_poly": (c_int, [V, V, c_longlong, V]),
     "krea2_attention_workspace_size": (c_size_t, [_PD, c_int, c_int, c_int, c_int]),
     "krea2_rope_tables": (c_int, [_PD, V, c_int, V, V, V]),
     "krea2_gqa_attention": (c_int, [_PD, c_int, c_int, c_int, c_int, V, V, V, V, V, V, V, V, c_size_t, V]),

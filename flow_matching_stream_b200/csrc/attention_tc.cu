@@ -26,8 +26,6 @@
 // prep kernel below does that once per element); v and gate are raw projection columns.
 #include <cuda.h>
 
-#include <algorithm>
-
 #include "krea2_device.cuh"
 #include "krea2_internal.h"
 
@@ -109,57 +107,6 @@ __device__ __forceinline__ float exp_tile(const float* v, float sl2, float m, ui
     float x0, x1;
     u2f(ffma2(f2u(v[2 * e], v[2 * e + 1]), s2, nm2), x0, x1);
     const float a = ex2(x0), c = ex2(x1);
-    pk[e] = pack_bf16x2(a, c);
-    acc[e & 3] = fadd2(acc[e & 3], f2u(a, c));
-  }
-  float t[8];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) u2f(acc[k], t[2 * k], t[2 * k + 1]);
-  return ((t[0] + t[1]) + (t[2] + t[3])) + ((t[4] + t[5]) + (t[6] + t[7]));
-}
-
-// 2^x on the FMA pipe, for x <= 8.5 (softmax arguments against a lazily raised running max).
-// x is clamped below at -125, split as x = n + f with n the nearest integer (adding 1.5 * 2^23
-// leaves n in the low mantissa bits) and f in [-1/2, 1/2]; 2^f is a cubic whose coefficients were
-// fitted by the Remez exchange algorithm for the smallest maximum relative error on that interval
-// (7.5e-5, against 2^-9 for the bf16 rounding of P); n is then added to the exponent field. The
-// clamp keeps that sum a normal number (at n = -126 a cubic value below 1 would fall into the
-// denormal range and lose its leading bit). Below the clamp the result is about 2^-125 instead of
-// 0, so tiles with masked keys (-inf scores) do not use it. Two values per call, on paired fp32
-// instructions.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  const unsigned long long magic = f2u(12582912.0f, 12582912.0f), nmagic = f2u(-12582912.0f, -12582912.0f);
-  const unsigned long long one_neg = f2u(-1.0f, -1.0f);
-  const unsigned long long x = f2u(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const unsigned long long t = fadd2(x, magic);        // n in the low bits of each mantissa
-  const unsigned long long f = ffma2(fadd2(t, nmagic), one_neg, x);  // x - n
-  unsigned long long q = ffma2(f2u(0.0551716685295105f, 0.0551716685295105f), f,
-                               f2u(0.2426111251115799f, 0.2426111251115799f));
-  q = ffma2(q, f, f2u(0.6932609677314758f, 0.6932609677314758f));
-  q = ffma2(q, f, f2u(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, t0, t1;
-  u2f(q, q0, q1);
-  u2f(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
-}
-
-// exp2 of (v * sl2 - m) for NE finite scores, one pair in POLY_EVERY through exp2_poly2 and the rest
-// on the MUFU; packed to bf16 pairs; returns the sum of the fp32 values.
-template <int NE, int POLY_EVERY>
-__device__ __forceinline__ float exp_tile_mixed(const float* v, float sl2, float m, uint32_t* pk) {
-  const unsigned long long s2 = f2u(sl2, sl2), nm2 = f2u(-m, -m);
-  unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-  for (int e = 0; e < NE / 2; ++e) {
-    float x0, x1, a, c;
-    u2f(ffma2(f2u(v[2 * e], v[2 * e + 1]), s2, nm2), x0, x1);
-    if (e % POLY_EVERY == POLY_EVERY - 1) {
-      exp2_poly2(x0, x1, a, c);
-    } else {
-      a = ex2(x0);
-      c = ex2(x1);
-    }
     pk[e] = pack_bf16x2(a, c);
     acc[e & 3] = fadd2(acc[e & 3], f2u(a, c));
   }
@@ -539,380 +486,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   }
 }
 
-// ============================================================================ two query tiles
-// One CTA per SM carries two 128-row query tiles (2 * 128/G positions of one KV head) that take
-// turns on the tensor pipe, over 128-key tiles:
-//   * TMEM (all 512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512). P_t is
-//     written as bf16 pairs over the first 64 columns of S_t and is the TMEM A operand of P_t V.
-//   * warp 0: TMA producer (both Q tiles once; K and V 128-key tiles, 2-stage rings, K tile i+1
-//     ahead of V tile i). No cluster multicast.
-//   * warp 1: MMA issuer. Per key tile i and query tile t it issues P_t V_{i-1} and then
-//     S_t = Q_t K_i^T (which overwrites P_{t,i-1}: MMAs of one thread execute in issue order).
-//     While one tile's softmax runs, the tensor pipe works on the other tile.
-//   * warps 2..5 (tile 0) and 6..9 (tile 1): one softmax thread per tile row (TMEM lane) holds
-//     all 128 scores, so the row max needs no exchange. s_full_t of tile i implies P_t V_{i-1}
-//     has run (it was issued before S_t), so a thread that raises its running max by more than
-//     2^8 rescales its O row right there, before it releases P_t.
-//   * shared memory: Q 64 KB, K and V 2 x 32 KB each; one CTA per SM.
-// Barrier phases: s_full[t], p_full[t] complete once per key tile, o_full[t] once at the end;
-// S_{t,i+1} is issued only after P_t V_i, which waits for every thread's P_{t,i}, so no thread
-// can be two phases behind a barrier it waits on.
-namespace two {
-constexpr int KT = 128;                 // keys per tile
-constexpr int STAGES = 2;               // K and V ring depth
-constexpr int THREADS = 320;            // producer, MMA issuer, 2 x 4 softmax warps
-constexpr int Q_CHUNK = 128 * 128;      // 128 rows x 64 bf16 (128 B) = 16 KB
-constexpr int Q_TILE = 2 * Q_CHUNK;     // 32 KB
-constexpr int KV_CHUNK = KT * 128;      // 128 keys x 128 B = 16 KB
-constexpr int KV_TILE = 2 * KV_CHUNK;   // 32 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + 2 * Q_TILE;
-constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
-constexpr int SMEM = OFF_V + STAGES * KV_TILE + 1024;  // 192 KB + alignment slack
-constexpr int MAX_TILES = 512;          // S <= 65536
-constexpr int POLY_EVERY = 4;           // in unmasked tiles one exp2 pair in 4 runs on the FMA pipe
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 2 * KT;
-constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, KT, 0, 0);
-constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, AD, 0, 1);
-}  // namespace two
-
-template <int G, bool PREFIX>
-__global__ void __launch_bounds__(two::THREADS, 1)
-    attn_gqa_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, AttnCore p) {
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t q_full;
-  __shared__ __align__(8) uint64_t k_full[two::STAGES];
-  __shared__ __align__(8) uint64_t v_full[two::STAGES];
-  __shared__ __align__(8) uint64_t k_empty[two::STAGES];  // freed when S_1 = Q_1 K^T (the tile's last read) is done
-  __shared__ __align__(8) uint64_t v_empty[two::STAGES];  // freed when P_1 V is done
-  __shared__ __align__(8) uint64_t s_full[2];        // per query tile: S_t of the current key tile
-  __shared__ __align__(8) uint64_t p_full[2];        // per query tile: all 128 rows wrote P_t
-  __shared__ __align__(8) uint64_t o_full[2];        // per query tile: the last P_t V is done
-  __shared__ __align__(8) uint64_t drain_bar;
-  __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag;
-  __shared__ int n_tiles;
-  __shared__ int cta_kmin;  // PREFIX: smallest key_end of this CTA's queries
-  __shared__ uint16_t tiles[two::MAX_TILES];
-
-  constexpr int QPOS = 128 / G;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p0 = blockIdx.x * (2 * QPOS), j = blockIdx.y, b = blockIdx.z;
-  const uint32_t base_u32 = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  uint8_t* base = smem_raw + (base_u32 - smem_u32(smem_raw));
-
-  // ---- key tiles holding at least one valid key (all-padded text tiles are skipped; with a key
-  // prefix, tiles at or beyond the largest key_end of the CTA's queries too)
-  if (warp == 0) {
-    int kmax = p.S;
-    if constexpr (PREFIX) {
-      int hi = 0, lo = p.S;
-      for (int i = lane; i < 2 * QPOS; i += 32) {
-        const int q = p0 + i;
-        if (q < p.Sq) {
-          const int e = min(max(p.key_end[q], p.q_off + q + 1), p.S);
-          hi = max(hi, e);
-          lo = min(lo, e);
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      }
-      kmax = hi;
-      if (lane == 0) cta_kmin = lo;
-    }
-    const int total = (min(kmax, p.S) + two::KT - 1) / two::KT;
-    int count = 0;
-    for (int t0 = 0; t0 < total; t0 += 32) {
-      const int t = t0 + lane;
-      bool valid = false;
-      if (t < total) {
-        const int k0 = t * two::KT;
-        const int k1 = min(k0 + two::KT, p.S);
-        if (!p.text_mask || k1 > p.T) {
-          valid = true;  // every key valid, or the tile holds image keys (always valid)
-        } else {
-          for (int k = k0; k < k1 && !valid; ++k) valid = p.text_mask[(long)b * p.T + k] != 0;
-        }
-      }
-      const unsigned m = __ballot_sync(0xffffffffu, valid);
-      if (valid) tiles[count + __popc(m & ((1u << lane) - 1u))] = (uint16_t)t;
-      count += __popc(m);
-    }
-    if (lane == 0) n_tiles = count;
-  }
-  if (threadIdx.x == 0) {
-    mbar_init(&q_full, 1);
-    for (int s = 0; s < two::STAGES; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
-    }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
-      mbar_init(&o_full[t], 1);
-    }
-    mbar_init(&drain_bar, 1);
-    abort_flag = 0;
-    fence_barrier_init();
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-  }
-  if (warp == 1) tmem_alloc(&tmem_slot, two::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_slot;
-  const int n = n_tiles;
-  volatile int* abort = &abort_flag;
-
-  if (warp == 0) {
-    if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(&q_full, 2 * two::Q_TILE);
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int hl = 0; hl < G; ++hl)
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            tma_load_3d(base + two::OFF_Q + t * two::Q_TILE + c * two::Q_CHUNK + hl * (QPOS * 128), &tmQ, &q_full,
-                        (j * G + hl) * AD + c * 64, p0 + t * QPOS, b);
-      IssuedFills k_fills, v_fills;
-      auto load_kv = [&](int i, const CUtensorMap* tm, uint64_t* full, uint64_t* empty, int off,
-                         IssuedFills& fills) -> bool {
-        const int st = i % two::STAGES;
-        const uint32_t ph = (i / two::STAGES) & 1;
-        if (!mbar_wait(&empty[st], ph ^ 1, abort)) return false;
-        uint8_t* d = base + off + st * two::KV_TILE;
-        const int t0 = tiles[i] * two::KT;
-        mbar_arrive_expect_tx(&full[st], two::KV_TILE);
-        tma_load_3d(d, tm, &full[st], j * AD, t0, b);
-        tma_load_3d(d + two::KV_CHUNK, tm, &full[st], j * AD + 64, t0, b);
-        fills.note(st, ph);
-        return true;
-      };
-      // K tile i+1 is issued before V tile i: K stages free up after Q_1 K^T, V stages only after
-      // P_1 V, so the K loads run a tile further ahead
-      if (load_kv(0, &tmK, k_full, k_empty, two::OFF_K, k_fills)) {
-        for (int i = 0; i < n; ++i) {
-          if (i + 1 < n && !load_kv(i + 1, &tmK, k_full, k_empty, two::OFF_K, k_fills)) break;
-          if (!load_kv(i, &tmV, v_full, v_empty, two::OFF_V, v_fills)) break;
-        }
-      }
-      if (*abort) {  // a wait expired: let the copies this thread issued land before the CTA exits
-        mbar_wait_drain(&q_full, 0);
-        k_fills.drain(k_full, two::STAGES);
-        v_fills.drain(v_full, two::STAGES);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0 && n > 0) {
-      // descriptors differ only in the start-address field (16-byte units): base plus constant
-      const uint64_t dq0 = smem_desc_sw128(smem_u32(base + two::OFF_Q), 16, 1024);
-      const uint64_t dk0 = smem_desc_sw128(smem_u32(base + two::OFF_K), 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(smem_u32(base + two::OFF_V), two::KV_CHUNK, 1024);
-      bool issued = false;
-      // O_t += P_t V_i: A = P_t in TMEM (bf16 pairs over S_t), B = V (MN-major)
-      auto issue_pv = [&](int t, int i) -> bool {
-        const int st = i % two::STAGES;
-        if (!mbar_wait(&p_full[t], i & 1, abort)) return false;
-        if (t == 0 && !mbar_wait(&v_full[st], (i / two::STAGES) & 1, abort)) return false;
-        tc_fence_after();
-        const uint64_t dv = dv0 + (uint64_t)(st * (two::KV_TILE >> 4));
-        const uint32_t pt = tmem + t * two::KT;
-#pragma unroll
-        for (int kk = 0; kk < two::KT / 16; ++kk)
-          tc_mma_bf16_ts(tmem + two::O_COL + t * AD, pt + kk * 8, dv + (uint64_t)(kk * 16 * 128 >> 4), two::IDESC_PV,
-                         (i > 0 || kk > 0) ? 1u : 0u);
-        issued = true;
-        if (t == 1) tc_commit(&v_empty[st]);
-        return true;
-      };
-      bool ok = mbar_wait(&q_full, 0, abort);
-      for (int i = 0; i < n && ok; ++i) {
-        const int st = i % two::STAGES;
-        if (!mbar_wait(&k_full[st], (i / two::STAGES) & 1, abort)) break;
-        tc_fence_after();
-        const uint64_t dk = dk0 + (uint64_t)(st * (two::KV_TILE >> 4));
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (i > 0 && !issue_pv(t, i - 1)) {
-            ok = false;
-            break;
-          }
-          const uint64_t dq = dq0 + (uint64_t)(t * (two::Q_TILE >> 4));
-#pragma unroll
-          for (int kk = 0; kk < AD / 16; ++kk) {
-            const uint32_t qo = (kk >> 2) * two::Q_CHUNK + (kk & 3) * 32;
-            const uint32_t ko = (kk >> 2) * two::KV_CHUNK + (kk & 3) * 32;
-            tc_mma_bf16(tmem + t * two::KT, dq + (uint64_t)(qo >> 4), dk + (uint64_t)(ko >> 4), two::IDESC_QK,
-                        kk > 0 ? 1u : 0u);
-          }
-          issued = true;
-          tc_commit(&s_full[t]);
-        }
-        if (ok) tc_commit(&k_empty[st]);
-      }
-      if (ok && !*abort) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!issue_pv(t, n - 1)) break;
-          tc_commit(&o_full[t]);
-        }
-      }
-      if (*abort && issued) {  // let every MMA already issued finish before TMEM is released
-        tc_commit(&drain_bar);
-        mbar_wait_drain(&drain_bar, 0);
-      }
-    }
-  } else {
-    // ---- softmax: warpgroup t = (warp - 2) / 4 owns query tile t; its thread of TMEM lane r holds
-    // tile row r = head j*G + r / QPOS at position p0 + t*QPOS + r % QPOS
-    const int t = (warp - 2) >> 2;
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + t * two::KT;
-    const uint32_t o_addr = tmem + lane_off + two::O_COL + t * AD;
-    const float sl2 = p.scale_log2;
-    const int pos = p0 + t * QPOS + r % QPOS;
-    const int h = j * G + r / QPOS;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    int row_kend = p.S;
-    if constexpr (PREFIX) row_kend = pos < p.Sq ? min(max(p.key_end[pos], p.q_off + pos + 1), p.S) : p.S;
-    for (int i = 0; i < n; ++i) {
-      if (!mbar_wait(&s_full[t], i & 1, abort)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const int k0 = tiles[i] * two::KT;
-      float v[two::KT];
-      tmem_ld128(s_addr, v);
-      bool masked = false;  // warp-uniform
-      if ((k0 < p.T && p.text_mask) || (k0 + two::KT > p.S)) {  // only partial tiles mask
-        masked = true;
-        uint32_t vm[two::KT / 32];
-#pragma unroll
-        for (int c = 0; c < two::KT / 32; ++c) vm[c] = __ballot_sync(0xffffffffu, key_valid(p, b, k0 + c * 32 + lane));
-#pragma unroll
-        for (int e = 0; e < two::KT; ++e)
-          if (!((vm[e >> 5] >> (e & 31)) & 1u)) v[e] = -INFINITY;
-      }
-      if constexpr (PREFIX) {
-        if (k0 + two::KT > cta_kmin) {  // warp-uniform; each row then cuts at its own key_end
-          masked = true;
-          const int lim = row_kend - k0;
-#pragma unroll
-          for (int e = 0; e < two::KT; ++e)
-            if (e >= lim) v[e] = -INFINITY;
-        }
-      }
-      // row max: chain k takes v[k], v[k + 8], ..., v[k + 120] with three-input maxes
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float a = v[k];
-#pragma unroll
-        for (int u = 1; u < 15; u += 2) a = fmax3(a, v[k + 8 * u], v[k + 8 * u + 8]);
-        m8[k] = fmaxf(a, v[k + 120]);
-      }
-      const float mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7]));
-      const float mnew = fmaxf(m, mx * sl2);
-      const bool grow = mnew > m + 8.0f;  // m = -inf until the row has seen a valid key
-      float alpha = 1.f;
-      if (grow) {
-        alpha = ex2(m - mnew);  // 0 on the row's first valid tile
-        m = mnew;
-      }
-      const bool any_grow = __any_sync(0xffffffffu, grow);
-      const float mu = m == -INFINITY ? 0.f : m;
-      float rs = 0.f;
-      if (masked) {  // -inf scores: the MUFU's exp2 returns exactly 0 for them
-#pragma unroll
-        for (int c = 0; c < two::KT / 32; ++c) {
-          uint32_t pk[16];
-          rs += exp_tile<32>(v + 32 * c, sl2, mu, pk);
-          tmem_st16(s_addr + c * 16, pk);  // P (bf16 pairs) over the tile's first 64 columns
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < two::KT / 32; ++c) {
-          uint32_t pk[16];
-          rs += exp_tile_mixed<32, two::POLY_EVERY>(v + 32 * c, sl2, mu, pk);
-          tmem_st16(s_addr + c * 16, pk);
-        }
-      }
-      l = l * alpha + rs;
-      if (i > 0 && any_grow) {
-        // O_t holds P_t V up to tile i-1 (issued before S_t of tile i, so done by s_full) and
-        // P_t V_i waits for this thread's p_full arrival: rescale the row now
-#pragma unroll 1
-        for (int c = 0; c < AD / 32; ++c) {
-          float o[32];
-          tmem_ld32(o_addr + c * 32, o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= alpha;
-          tmem_st32(o_addr + c * 32, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
-    const bool row_ok = pos < p.Sq;
-    const long grow_idx = (long)b * p.Sq + pos;
-    if (ok && n == 0) {
-      // a batch row without any valid key (possible only without image tokens): zeros
-      if (row_ok) {
-        uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD);
-#pragma unroll
-        for (int q = 0; q < AD / 8; ++q) op[q] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    } else if (ok && mbar_wait(&o_full[t], 0, abort)) {
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;  // a row with no readable key: zeros
-#pragma unroll 1
-      for (int c = 0; c < AD / 32; ++c) {
-        float o[32];
-        tmem_ld32(o_addr + c * 32, o);
-        if (row_ok) {
-          const uint4* gp = reinterpret_cast<const uint4*>(p.gate + grow_idx * p.g_stride + h * AD + c * 32);
-          uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD + c * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 gv = __ldg(gp + q);
-            const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-            uint32_t ow[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float a = o[q * 8 + 2 * e] * inv_l * sigmoid_f(bf16_lo(gw[e]));
-              const float bb = o[q * 8 + 2 * e + 1] * inv_l * sigmoid_f(bf16_hi(gw[e]));
-              ow[e] = pack_bf16x2(a, bb);
-            }
-            op[q] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-          }
-        }
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, two::TMEM_COLS);
-  }
-}
-
 // One warp normalises one 128-wide head (RMSNorm over head_dim with weight (1 + w), page §四.3)
 // and rotates it by the position's RoPE angles (adjacent pairs); each lane holds 4 columns.
 __device__ __forceinline__ uint2 norm_rope_head(const __nv_bfloat16* x, const float* w, const float* cs,
@@ -1001,23 +574,6 @@ int launch_wait_timeout_selftest(unsigned long long limit_ns, int* waited, cudaS
   return KREA2_OK;
 }
 
-namespace {
-// y = exp2_poly2(x) elementwise (n even), for the numerics test of the polynomial.
-__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
-  for (long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x); i + 1 < n;
-       i += 2LL * gridDim.x * blockDim.x)
-    exp2_poly2(x[i], x[i + 1], y[i], y[i + 1]);
-}
-}  // namespace
-
-int launch_exp2_poly_selftest(const float* x, float* y, long long n, cudaStream_t stream) {
-  exp2_poly_selftest_kernel<<<(unsigned)std::min<long long>((n / 2 + 255) / 256, 4096), 256, 0, stream>>>(x, y, n);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "exp2 self-test launch failed: %s", cudaGetErrorString(e));
-  return KREA2_OK;
-}
-
 bool attention_tc_supported(int D, int H, int Hkv) {
   if (D != AD || Hkv <= 0 || H % Hkv) return false;
   const int g = H / Hkv;
@@ -1067,61 +623,19 @@ int launch_attention_g(const AttnTcArgs& a, cudaStream_t stream) {
 }
 }  // namespace
 
-namespace {
-template <int G, bool PREFIX>
-int launch_attention2_g(const AttnTcArgs& a, cudaStream_t stream) {
-  constexpr int QPOS = 128 / G;
-  auto kern = attn_gqa_tc2_kernel<G, PREFIX>;
-  static std::atomic<uint64_t> attr_done{0};
-  const uint64_t dev_bit = device_bit();
-  if (!(attr_done.load(std::memory_order_acquire) & dev_bit) || !dev_bit) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, two::SMEM) != cudaSuccess)
-      return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(attention) failed");
-    attr_done.fetch_or(dev_bit, std::memory_order_release);
-  }
-  const int S = a.T + a.N;
-  const int Sq = a.Sq > 0 ? a.Sq : S;
-  const long long kv_rows = a.kv_batch_rows > 0 ? a.kv_batch_rows : S;
-  if ((S + two::KT - 1) / two::KT > two::MAX_TILES)
-    return set_error(KREA2_ERR_UNSUPPORTED, "sequence longer than %d", two::MAX_TILES * two::KT);
-  if (Sq > S || a.q_off < 0 || a.q_off + Sq > S)
-    return set_error(KREA2_ERR_ARG, "query rows [%d, %d) lie outside the %d keys", a.q_off, a.q_off + Sq, S);
-  CUtensorMap tq, tk, tv;
-  int rc;
-  if ((rc = make_tmap_bf16_3d(&tq, a.q, (uint64_t)a.H * AD, Sq, a.B, a.q_stride, 64, QPOS, Sq))) return rc;
-  if ((rc = make_tmap_bf16_3d(&tk, a.k, (uint64_t)a.Hkv * AD, S, a.B, a.k_stride, 64, two::KT, kv_rows))) return rc;
-  if ((rc = make_tmap_bf16_3d(&tv, a.v, (uint64_t)a.Hkv * AD, S, a.B, a.v_stride, 64, two::KT, kv_rows))) return rc;
-  AttnCore p{};
-  p.B = a.B; p.T = a.T; p.N = a.N; p.S = S; p.Hkv = a.Hkv; p.HD = a.H * AD;
-  p.Sq = Sq; p.q_off = a.q_off;
-  p.text_mask = a.text_mask;
-  p.gate = reinterpret_cast<const __nv_bfloat16*>(a.g);
-  p.g_stride = a.g_stride;
-  p.out = reinterpret_cast<__nv_bfloat16*>(a.out);
-  p.scale_log2 = 1.4426950408889634f / sqrtf((float)AD);
-  p.key_end = a.key_end;
-  dim3 grid((Sq + 2 * QPOS - 1) / (2 * QPOS), a.Hkv, a.B);
-  kern<<<grid, two::THREADS, two::SMEM, stream>>>(tq, tk, tv, p);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "attention launch failed: %s", cudaGetErrorString(e));
-  return KREA2_OK;
-}
-}  // namespace
-
 int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream) {
   if (!attention_tc_supported(AD, a.H, a.Hkv)) return set_error(KREA2_ERR_UNSUPPORTED, "attention group size");
   if (a.key_end) {
     switch (a.H / a.Hkv) {
-      case 1: return launch_attention2_g<1, true>(a, stream);
-      case 2: return launch_attention2_g<2, true>(a, stream);
-      default: return launch_attention2_g<4, true>(a, stream);
+      case 1: return launch_attention_g<1, true>(a, stream);
+      case 2: return launch_attention_g<2, true>(a, stream);
+      default: return launch_attention_g<4, true>(a, stream);
     }
   }
   switch (a.H / a.Hkv) {
-    case 1: return launch_attention2_g<1, false>(a, stream);
-    case 2: return launch_attention2_g<2, false>(a, stream);
-    default: return launch_attention2_g<4, false>(a, stream);
+    case 1: return launch_attention_g<1, false>(a, stream);
+    case 2: return launch_attention_g<2, false>(a, stream);
+    default: return launch_attention_g<4, false>(a, stream);
   }
 }
 

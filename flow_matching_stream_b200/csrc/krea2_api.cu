@@ -292,11 +292,12 @@ int krea2_check_device_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));
   if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "stream error: %s", cudaGetErrorString(e));
   const int ve[2] = {take_device_error_gemm(), take_device_error_attention()};
+  const char* names[2] = {"GEMM", "attention"};
   for (int i = 0; i < 2; ++i) {
     if (ve[i] < 0) return set_error(KREA2_ERR_CUDA, "cannot read the device error word");
     if (ve[i] > 0)
       return set_error(KREA2_ERR_TIMEOUT, "a bounded device-side wait expired in the %s kernels (code %d)",
-                       i == 0 ? "GEMM" : "attention", ve[i]);
+                       names[i], ve[i]);
   }
   return KREA2_OK;
 }
@@ -304,12 +305,6 @@ int krea2_check_device_error(void* stream) {
 int krea2_selftest_wait_timeout(int limit_ms, int* waited, void* stream) {
   if (limit_ms < 1 || limit_ms > 5000 || !waited) return set_error(KREA2_ERR_ARG, "limit_ms must be 1..5000, waited non-NULL");
   return launch_wait_timeout_selftest((unsigned long long)limit_ms * 1000000ull, waited, as_stream(stream));
-}
-
-int krea2_selftest_exp2_poly(const float* x, float* y, long long n, void* stream) {
-  if (!x || !y || n < 0 || (n & 1)) return set_error(KREA2_ERR_ARG, "need x, y non-NULL and an even n >= 0");
-  if (n == 0) return KREA2_OK;
-  return launch_exp2_poly_selftest(x, y, n, as_stream(stream));
 }
 
 size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype) {

@@ -225,30 +225,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
       : "memory");
 }
 
-// 128 consecutive fp32 columns of the thread's lane in one load, under the same wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
-  uint32_t* r = reinterpret_cast<uint32_t*>(v);
-#define KREA2_R8(b) \
-  "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), "=r"(r[b + 6]), "=r"(r[b + 7])
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
-      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, "
-      "%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
-      "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
-      "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
-      "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%128];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : KREA2_R8(0), KREA2_R8(8), KREA2_R8(16), KREA2_R8(24), KREA2_R8(32), KREA2_R8(40), KREA2_R8(48),
-        KREA2_R8(56), KREA2_R8(64), KREA2_R8(72), KREA2_R8(80), KREA2_R8(88), KREA2_R8(96), KREA2_R8(104),
-        KREA2_R8(112), KREA2_R8(120)
-      : "r"(taddr)
-      : "memory");
-#undef KREA2_R8
-}
-
 // Each thread of the warp writes 32 consecutive fp32 columns of its TMEM lane.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
   const uint32_t* r = reinterpret_cast<const uint32_t*>(v);

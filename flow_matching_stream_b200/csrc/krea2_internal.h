@@ -142,7 +142,6 @@ struct AttnTcArgs {
 };
 bool attention_tc_supported(int D, int H, int Hkv);
 int launch_wait_timeout_selftest(unsigned long long limit_ns, int* waited, cudaStream_t stream);
-int launch_exp2_poly_selftest(const float* x, float* y, long long n, cudaStream_t stream);
 int attention_tc_core(const AttnTcArgs& a, cudaStream_t stream);
 // raw k and v of n tokens -> rows [row0, row0 + n) of every batch row of a key/value cache
 // (k RMS-normalised and rotated, v copied; bf16, (B, capacity, Hkv*128))

@@ -128,13 +128,6 @@ int krea2_check_device_error(void* stream);
  * KREA2_ERR_TIMEOUT and clears the error word. The context stays usable. */
 int krea2_selftest_wait_timeout(int limit_ms, int* waited, void* stream);
 
-/* Numerics self-test of the attention kernel's exp2 on the FMA pipe (no counterpart in the pages:
- * the softmax of [ARCH] §四.3 needs exp, and the tensor-core attention evaluates some of its
- * exponentials with a cubic instead of the MUFU). x, y: n fp32 DEVICE values, n even; writes
- * y[i] ~ 2^x[i] for x[i] in [-125, 8.5] with at most 7.5e-5 relative error (the fit's bound);
- * below -125 the result is about 2^-125. KREA2_ERR_ARG for odd n or NULL pointers. */
-int krea2_selftest_exp2_poly(const float* x, float* y, long long n, void* stream);
-
 /* Bytes of device workspace that krea2_block_forward / krea2_backbone_forward need for
  * these shapes (0 on invalid arguments). The workspace must be 256-byte aligned. */
 size_t krea2_workspace_size(const Krea2Dims* dims, int B, int T, int N, int dtype);

@@ -81,9 +81,9 @@ def test_linear_gated_residual(K2, B, S, N, K):
 
 @pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, 8e-3), (torch.float32, 1e-5)])
 @pytest.mark.parametrize("chunk", [0, 3])
-def test_modulated_rmsnorm(K2, dtype, tol, chunk):
+@pytest.mark.parametrize("B,S", [(2, 333), (2, 1500)])
+def test_modulated_rmsnorm(K2, dtype, tol, chunk, B, S):
     d = KI.FULL
-    B, S = 2, 333
     h = KI.residual(d, B, S)
     temb = KI.temb(d, B)
     table = KI._normal(0, (99, 1), (6, d.C), 0.1)
@@ -125,36 +125,3 @@ def test_final_layer(K2, dims, dtype, tol):
     K2.final_layer(dims, B, T, N, dev(h.reshape(B * S, dims.C), torch.float32), dev(e, torch.float32), mw, vel, ws)
     ref = O.final_layer(h[:, T:], e, mw_h, dims.eps)
     assert rel_err(host(vel).reshape(B, N, dims.in_ch), ref) < tol
-
-
-def test_exp2_polynomial_against_cuda_exp2f(cuda_device):
-    # the attention kernel evaluates some softmax exponentials with a fitted cubic on the FMA pipe:
-    # relative error at most 7.5e-5 (the fit's bound) over its range, against torch.exp2 (CUDA's
-    # exp2f) and against fp64
-    import ctypes
-    import flow_matching_stream_b200 as K2
-    lib = K2.lib()
-    x = torch.cat([torch.linspace(-125.0, 8.5, 1 << 20, device="cuda"),
-                   torch.rand(1 << 20, device="cuda", generator=torch.Generator(device="cuda").manual_seed(0)) * 40 - 32,
-                   torch.arange(-125, 9, device="cuda", dtype=torch.float32),
-                   torch.arange(-125, 8, device="cuda", dtype=torch.float32) + 0.5])
-    x = x[: x.numel() // 2 * 2].contiguous()
-    y = torch.empty_like(x)
-    stream = torch.cuda.current_stream().cuda_stream
-    assert lib.krea2_selftest_exp2_poly(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), x.numel(),
-                                        stream) == 0
-    assert lib.krea2_check_device_error(stream) == 0
-    ref32 = torch.exp2(x)
-    rel = ((y - ref32).abs() / ref32).max().item()
-    ref64 = torch.exp2(x.double())
-    rel64 = ((y.double() - ref64).abs() / ref64).max().item()
-    print(f"exp2 polynomial: max rel err {rel:.3e} vs exp2f, {rel64:.3e} vs fp64")
-    assert rel < 8e-5 and rel64 < 8e-5
-    # below the clamp: about 2^-125, finite and non-negative, never NaN
-    lo = torch.tensor([-125.4, -126.0, -130.0, -1e4, float("-inf"), -125.0], device="cuda")
-    ylo = torch.empty_like(lo)
-    assert lib.krea2_selftest_exp2_poly(ctypes.c_void_p(lo.data_ptr()), ctypes.c_void_p(ylo.data_ptr()), 6,
-                                        stream) == 0
-    torch.cuda.synchronize()
-    assert torch.all(torch.isfinite(ylo)) and torch.all(ylo > 0) and torch.all(ylo < 4e-38)
-    assert lib.krea2_selftest_exp2_poly(None, None, 3, None) == -1

@@ -182,8 +182,6 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
 }
 
 // out[b, n] = act(sum_k x[b, k] W[n, k] + bias[n]); one warp per output feature, all batch rows.
-// The K loop is unrolled by 4 so that each lane keeps four 16-byte weight loads in flight: the
-// weights stream from HBM once per forward and this kernel is bound by that stream.
 template <bool W_BF16, bool GELU>
 __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __restrict__ x, const void* __restrict__ W,
                                                              const float* __restrict__ bias, int B, int N, int K,
@@ -196,7 +194,6 @@ __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __rest
     float acc[MAXB];
 #pragma unroll
     for (int b = 0; b < MAXB; ++b) acc[b] = 0.f;
-#pragma unroll 4
     for (int k = lane * 8; k < K; k += 256) {
       float wv[8];
       if (W_BF16) {

@@ -290,8 +290,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       auto issue_pv = [&](int i) -> bool {
         // O += P_i V_i : A = P_i in TMEM (bf16 pairs over its scores), B = V (MN-major)
         const int st = i % KV_STAGES;
-        if (!mbar_wait(&p_full[i & 1], (i >> 1) & 1, abort)) return false;
-        if (!mbar_wait(&v_full[st], (i / KV_STAGES) & 1, abort)) return false;
+        // P_i and V_i: both tests go out together (the V load has usually landed long before)
+        if (!mbar_wait2(&p_full[i & 1], (i >> 1) & 1, &v_full[st], (i / KV_STAGES) & 1, abort)) return false;
         tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)(st * (KV_TILE_BYTES >> 4));
         const uint32_t pt = tmem + (i & 1) * KT;

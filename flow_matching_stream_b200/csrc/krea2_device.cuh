@@ -88,6 +88,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits for two barrier phases. Both are first tested back to back, without blocking, so that
+// when both are already complete (the common case for one of them) the two latencies overlap.
+__device__ __forceinline__ bool mbar_wait2(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb, volatile int* abort) {
+  uint32_t oka, okb;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%2], %3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q, [%4], %5;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "selp.u32 %1, 1, 0, q;\n\t}"
+      : "=r"(oka), "=r"(okb)
+      : "r"(smem_u32(a)), "r"(pa), "r"(smem_u32(b)), "r"(pb)
+      : "memory");
+  if (oka && okb) return true;
+  return (oka || mbar_wait(a, pa, abort)) && (okb || mbar_wait(b, pb, abort));
+}
+
 // Waits up to limit_ns for the phase of the given parity to complete, whatever the abort flag
 // says. The abort path uses it so that TMA copies already issued into shared memory land before
 // the CTA exits.

@@ -23,6 +23,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
+
 #include "krea2_device.cuh"
 #include "krea2_internal.h"
 
@@ -32,9 +34,9 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-// Row tiles per raster group: as many as keep the group's A tiles (128 x K bf16 each) within
-// about 24 MB of L2, so W streams from HBM once per group pass. Larger groups measured more
-// DRAM re-reads of W, not fewer: their A tiles did not stay resident.
+// Row tiles per raster group (group_rows below): at least as many as keep the group's A tiles
+// (128 x K bf16 each) within about 24 MB of L2, so W streams from HBM once per group pass, and
+// at least as many as make one wave of tiles read about as many A bytes as W bytes per K step.
 constexpr size_t GROUP_A_BYTES = 24ull << 20;
 constexpr int GEMM_THREADS = 192;
 
@@ -451,6 +453,20 @@ int make_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
 
 namespace {
 
+// Row tiles per raster group. The persistent CTAs run about `sms` consecutive tiles at once: r
+// row tiles by c = sms / r column tiles of one group. Per K step that wave reads r*BM rows of A
+// and c*BN rows of W, which is least at r = sqrt(sms * BN / BM) (18 for BN = 256 on 148 SMs);
+// fewer rows stream W from HBM once per wave (down, K = 16384, took 6 by the L2 rule alone).
+// The row tiles are then split into groups of equal size.
+int group_rows(int tiles_m, int K, int BN, int sms) {
+  const int by_l2 = (int)(GROUP_A_BYTES / ((size_t)BM * K * 2));
+  const int by_wave = (int)std::ceil(std::sqrt((double)sms * BN / BM));
+  int g = by_l2 > by_wave ? by_l2 : by_wave;
+  if (g >= tiles_m) return tiles_m;
+  const int groups = (tiles_m + g - 1) / g;
+  return (tiles_m + groups - 1) / groups;
+}
+
 template <int BN, int EPI>
 int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
@@ -470,12 +486,7 @@ int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStrea
   GemmParams p = p0;
   p.tiles_m = (p.M + BM - 1) / BM;
   p.tiles_n = p.N / BN;
-  {
-    const size_t per_tile = (size_t)BM * p.K * 2;
-    int g = (int)(GROUP_A_BYTES / per_tile);
-    g = g < 8 ? 8 : g;
-    p.group_m = g < p.tiles_m ? g : p.tiles_m;
-  }
+  p.group_m = group_rows(p.tiles_m, p.K, BN, num_sms());
   const int total = p.tiles_m * p.tiles_n;
   const int grid = total < num_sms() ? total : num_sms();
   kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);

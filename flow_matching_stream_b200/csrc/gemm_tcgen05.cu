@@ -24,6 +24,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstring>
 
 #include "krea2_device.cuh"
 #include "krea2_internal.h"
@@ -46,8 +47,11 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN=256) or 16 KB (BN=128)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr int XPOSE_BYTES = 4 * 32 * 33 * 4;  // residual epilogue: one padded 32x32 fp32 tile per warp
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + XPOSE_BYTES + 1024;  // + alignment slack
+  // Epilogue staging per warp: two 4 KB swizzled 32x32 fp32 boxes (residual), or one padded
+  // 32x33 fp32 tile (the other epilogues), at 8 KB spacing.
+  static constexpr int EPI_WARP_BYTES = 8192;
+  static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 2 * BN;                         // double-buffered fp32
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 };
@@ -65,26 +69,45 @@ struct TileMap {
   }
 };
 
-// Each thread holds 32 consecutive bf16 pairs (64 columns) of its accumulator row. The warp
-// writes its 32 rows through a padded shared tile, so every global store covers 128 bytes of
-// one row instead of 16 bytes of each of 32 rows.
-__device__ __forceinline__ void store_bf16_rows(uint32_t* xp, const uint32_t* pk, __nv_bfloat16* dst0, size_t ld,
-                                                int nrows, int lane) {
+// The TMA epilogues hand each warp's 32 rows to the TMA unit through boxes in shared memory:
+// 32 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle, so 16-byte chunk j of box
+// row r sits at position j ^ (r & 7) and a warp's row-wise 16-byte stores spread over all banks.
+// Rows and columns outside the output are clipped by the tensor map. Each warp owns two boxes
+// and alternates between them; a box is rewritten only once the TMA operation issued from it two
+// boxes earlier has finished reading it.
+struct EpiBoxes {
+  uint8_t* smem;
+  int n;
+  __device__ __forceinline__ uint8_t* next(int lane) {
+    uint8_t* b = smem + (n++ & 1) * 4096;
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+    return b;
+  }
+};
+
+__device__ __forceinline__ void box_put16(uint8_t* box, int lane, int j, uint4 v) {
+  *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+}
+
+// Thread `lane` holds row `lane` of a 32 x 64 bf16 block as 32 packed pairs; the warp stores the
+// block at output column x, row y (issue = false skips a block wholly past the last row).
+__device__ __forceinline__ void store_box_bf16(uint8_t* box, const uint32_t* pk, int lane, const CUtensorMap* tm,
+                                               int x, int y, bool issue) {
 #pragma unroll
-  for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = pk[e];
+  for (int j = 0; j < 8; ++j) box_put16(box, lane, j, make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]));
+  fence_proxy_async_smem();
   __syncwarp();
-  uint32_t* d = reinterpret_cast<uint32_t*>(dst0) + lane;
-  const size_t ldw = ld / 2;  // row stride in bf16 pairs
-#pragma unroll 8
-  for (int i = 0; i < 32; ++i)
-    if (i < nrows) d[(size_t)i * ldw] = xp[i * 33 + lane];
-  __syncwarp();
+  if (lane == 0 && issue) {
+    tma_store_2d(tm, box, x, y);
+    bulk_commit_group();
+  }
 }
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             GemmParams p) {
+                             const __grid_constant__ CUtensorMap tmC, GemmParams p) {
   using Cfg = GemmCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
 
@@ -200,6 +223,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else {
     // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
     const int quarter = warp & 3;
+    EpiBoxes boxes{base + STAGES * Cfg::STAGE_BYTES + (warp - 2) * Cfg::EPI_WARP_BYTES, 0};
     int local = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
       int mt, nt;
@@ -214,11 +238,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
       const int row0 = mt * BM + quarter * 32;
       const int nrows = min(32, p.M - row0);
-      uint32_t* xpk = reinterpret_cast<uint32_t*>(base + STAGES * Cfg::STAGE_BYTES) + (warp - 2) * (32 * 33);
+      uint8_t* epi_smem = base + STAGES * Cfg::STAGE_BYTES + (warp - 2) * Cfg::EPI_WARP_BYTES;
+      uint32_t* xpk = reinterpret_cast<uint32_t*>(epi_smem);
+      const bool rows_in = row0 < p.M;  // warp-uniform: this 32-row block holds output rows
       if constexpr (EPI == EPI_STORE) {
-        const int ld = p.out_ld ? p.out_ld : p.N;
         const int n_store = p.n_store ? p.n_store : p.N;
-        __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row0 * ld + (size_t)nt * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 64; ++c) {
           if (nt * BN + c * 64 >= n_store) break;  // warp-uniform: padding columns of W are not stored
@@ -238,7 +262,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-          store_bf16_rows(xpk, pk, out0 + c * 64, ld, nrows, lane);
+          store_box_bf16(boxes.next(lane), pk, lane, &tmC, nt * BN + c * 64, row0, rows_in);
         }
       } else if constexpr (EPI == EPI_BIAS_ROWMAP) {
         // fp32 out[map(row), col] = acc + bias[col], rows transposed through shared memory like the
@@ -264,37 +288,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           __syncwarp();
         }
       } else if constexpr (EPI == EPI_SWIGLU) {
-        // interleaved 64-row groups: columns [128g, 128g+64) gate, [128g+64, 128g+128) up
-        const int ldo = p.N / 2;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row * ldo + (size_t)nt * (BN / 2);
+        // interleaved 64-row groups: columns [128g, 128g+64) gate, [128g+64, 128g+128) up; each
+        // group gives 64 output columns
 #pragma unroll 1
         for (int g = 0; g < BN / 128; ++g) {
-#pragma unroll 1
+          uint32_t pk[32];
+#pragma unroll
           for (int half = 0; half < 2; ++half) {
             float gv[32], uv[32];
             tmem_ld32(tbase + g * 128 + half * 32, gv);
             tmem_ld32(tbase + g * 128 + 64 + half * 32, uv);
-            if (row_ok) {
-              uint4* dst = reinterpret_cast<uint4*>(out + g * 64 + half * 32);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                float r[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) r[e] = silu_f(gv[q * 8 + e]) * uv[q * 8 + e];
-                uint4 w;
-                w.x = pack_bf16x2(r[0], r[1]);
-                w.y = pack_bf16x2(r[2], r[3]);
-                w.z = pack_bf16x2(r[4], r[5]);
-                w.w = pack_bf16x2(r[6], r[7]);
-                dst[q] = w;
-              }
-            }
+            for (int e = 0; e < 16; ++e)
+              pk[half * 16 + e] = pack_bf16x2(silu_f(gv[2 * e]) * uv[2 * e], silu_f(gv[2 * e + 1]) * uv[2 * e + 1]);
           }
+          store_box_bf16(boxes.next(lane), pk, lane, &tmC, nt * (BN / 2) + g * 64, row0, rows_in);
         }
       } else if constexpr (EPI == EPI_QKV) {
         // [q | k | v | gate] columns; 128-wide q/k heads get RMSNorm (1 + w) and RoPE here,
         // once per element, on the fp32 accumulator (page §四.3 order: norm, then RoPE)
-        __nv_bfloat16* out0 = reinterpret_cast<__nv_bfloat16*>(p.out) + (size_t)row0 * p.N + (size_t)nt * BN;
         const int pos = row_ok ? row % p.rows_per_batch : 0;
         const float* cs = p.cos + (size_t)pos * 64;
         const float* sn = p.sin + (size_t)pos * 64;
@@ -343,48 +355,55 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             uint32_t pk[32];
 #pragma unroll
             for (int e = 0; e < 32; ++e) pk[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-            store_bf16_rows(xpk, pk, out0 + u * 128 + h2 * 64, p.N, nrows, lane);
+            store_box_bf16(boxes.next(lane), pk, lane, &tmC, nt * BN + u * 128 + h2 * 64, row0, rows_in);
           }
         }
       } else {  // EPI_RESID: h[row, col] += gate[b, col] * acc
-        // After tcgen05.ld each thread holds one row of a 32-column chunk. Read-modify-write of
-        // the fp32 residual row by row would make every warp access touch 32 cache lines (one
-        // L1 wavefront each, in the SRAM that also feeds the tensor core), so the warp
-        // transposes its 32x32 block through a padded shared tile and then walks the rows: each
-        // access is one 128-byte line, and 16 rows of loads are in flight before any store.
-        // Lane i knows the batch row of tile row row0 + i (clamped to M - 1, so that rows of the
-        // ragged last tile read an in-bounds gate; their results are never stored).
-        float* xp = reinterpret_cast<float*>(xpk);
+        // Each thread scales its row of a 32-column chunk by the gate of its batch row and
+        // writes it into a 32x32 fp32 box; one lane hands the box to the TMA unit as a
+        // reduce-add into h. The read-modify-write of the residual then runs in L2, and the
+        // epilogue never waits on loads of h. The batch row of a ragged last tile's rows is
+        // clamped to M - 1 (an in-bounds gate; those rows are clipped by the tensor map).
         const int my_b = min(row0 + lane, p.M - 1) / p.rows_per_batch;
+        const float* grow = p.gate + (size_t)my_b * p.gate_stride + (size_t)nt * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
+          uint8_t* box = boxes.next(lane);
+          if (p.gate_vec4) {
+            const float4* g4 = reinterpret_cast<const float4*>(grow + c * 32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = v[e];
-          __syncwarp();
-          const int col = nt * BN + c * 32 + lane;
-#pragma unroll 1
-          for (int i0 = 0; i0 < 32; i0 += 16) {
-            float* hp = reinterpret_cast<float*>(p.out) + (size_t)(row0 + i0) * p.N + col;
-            float hv[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) hv[i] = i0 + i < nrows ? hp[(size_t)i * p.N] : 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int bb = __shfl_sync(0xffffffffu, my_b, i0 + i);
-              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
+            for (int j = 0; j < 8; ++j) {
+              const float4 g = __ldg(g4 + j);
+              box_put16(box, lane, j,
+                        make_uint4(__float_as_uint(v[4 * j] * g.x), __float_as_uint(v[4 * j + 1] * g.y),
+                                   __float_as_uint(v[4 * j + 2] * g.z), __float_as_uint(v[4 * j + 3] * g.w)));
             }
+          } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (i0 + i < nrows) hp[(size_t)i * p.N] = hv[i];
+            for (int j = 0; j < 8; ++j) {
+              const float* gj = grow + c * 32 + 4 * j;
+              box_put16(box, lane, j,
+                        make_uint4(__float_as_uint(v[4 * j] * __ldg(gj)), __float_as_uint(v[4 * j + 1] * __ldg(gj + 1)),
+                                   __float_as_uint(v[4 * j + 2] * __ldg(gj + 2)),
+                                   __float_as_uint(v[4 * j + 3] * __ldg(gj + 3))));
+            }
           }
+          fence_proxy_async_smem();
           __syncwarp();
+          if (lane == 0 && rows_in) {  // a 32-row block wholly past M (ragged last tile) adds nothing
+            tma_reduce_add_2d(&tmC, box, nt * BN + c * 32, row0);
+            bulk_commit_group();
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
     }
+    // the TMA stores and reduces must be complete (their boxes read, the output written) before
+    // this CTA's shared memory goes away
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncthreads();
@@ -424,6 +443,23 @@ int make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return KREA2_OK;
+}
+
+// Row-major fp32 matrix (rows, cols) as a 2-D TMA map with a 32x32 box and 128-byte swizzle: the
+// residual epilogue's reduce-add target.
+static int make_tmap_f32_2d_box32(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((cols * 4) & 15))
+    return set_error(KREA2_ERR_ARG, "residual output must be 16-byte aligned with a 16-byte multiple row stride");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled (fp32) failed (%d)", (int)r);
   return KREA2_OK;
 }
 
@@ -478,18 +514,31 @@ int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStrea
       return set_error(KREA2_ERR_CUDA, "cudaFuncSetAttribute(gemm) failed");
     attr_done.fetch_or(dev_bit, std::memory_order_release);
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   int rc = make_tmap_bf16_2d(&ta, A, p0.K, p0.M, p0.K, BK, BM);
   if (rc) return rc;
   rc = make_tmap_bf16_2d(&tb, W, p0.K, p0.w_rows ? p0.w_rows : p0.N, p0.K, BK, BN);
   if (rc) return rc;
   GemmParams p = p0;
+  // the epilogue's TMA target: 32-row boxes of 128 bytes (64 bf16 or 32 fp32 columns)
+  memset(&tc, 0, sizeof(tc));
+  if constexpr (EPI == EPI_RESID) {
+    if ((rc = make_tmap_f32_2d_box32(&tc, p.out, p.N, p.M))) return rc;
+    p.gate_vec4 = !(reinterpret_cast<uintptr_t>(p.gate) & 15) && !(p.gate_stride & 3);
+  } else if constexpr (EPI == EPI_STORE) {
+    if ((rc = make_tmap_bf16_2d(&tc, p.out, p.n_store ? p.n_store : p.N, p.M, p.out_ld ? p.out_ld : p.N, 64, 32)))
+      return rc;
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    if ((rc = make_tmap_bf16_2d(&tc, p.out, p.N / 2, p.M, p.N / 2, 64, 32))) return rc;
+  } else if constexpr (EPI == EPI_QKV) {
+    if ((rc = make_tmap_bf16_2d(&tc, p.out, p.N, p.M, p.N, 64, 32))) return rc;
+  }
   p.tiles_m = (p.M + BM - 1) / BM;
   p.tiles_n = p.N / BN;
   p.group_m = group_rows(p.tiles_m, p.K, BN, num_sms());
   const int total = p.tiles_m * p.tiles_n;
   const int grid = total < num_sms() ? total : num_sms();
-  kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, p);
+  kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, tc, p);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "gemm launch failed: %s", cudaGetErrorString(e));

@@ -39,44 +39,81 @@ def _bf(shape, seed, scale=1.0):
 @pytest.mark.parametrize("M,N,K", [(300, 512, 256), (1152, 6144, 6144), (129, 384, 640), (1, 128, 64)])
 def test_linear_store(K2, M, N, K):
     A, W = _bf((M, K), 1), _bf((N, K), 2, K ** -0.5)
-    out = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    # the output is the first M rows of a buffer whose 40 sentinel rows must stay untouched
+    buf = torch.full((M + 40, N), 7.0, device="cuda", dtype=torch.bfloat16)
+    out = buf[:M]
     K2.linear(K2.KREA2_EPI_STORE, dev(A, torch.bfloat16), dev(W, torch.bfloat16), out)
     K2.check_device_error()
     ref = A @ W.T  # fp32 BLAS: ~1e-6 relative, far below the bf16 output rounding
     assert rel_err(host(out), ref) < 8e-3
+    assert torch.all(buf[M:] == 7.0).item()
+
+
+def test_linear_store_unaligned_out_rejected(K2):
+    """Outputs are written by TMA stores, which need a 16-byte aligned base address."""
+    M, N, K = 64, 128, 64
+    A, W = _bf((M, K), 1), _bf((N, K), 2, K ** -0.5)
+    buf = torch.zeros(M * N + 1, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(K2.Krea2Error):
+        K2.linear(K2.KREA2_EPI_STORE, dev(A, torch.bfloat16), dev(W, torch.bfloat16), buf[1:].view(M, N))
+    K2.check_device_error()
+    assert torch.count_nonzero(buf).item() == 0
 
 
 @pytest.mark.parametrize("M,F,K", [(200, 256, 128), (1152, 16384, 6144)])
 def test_linear_swiglu(K2, M, F, K):
     A, Wg, Wu = _bf((M, K), 3), _bf((F, K), 4, K ** -0.5), _bf((F, K), 5, K ** -0.5)
     Wgu = K2.interleave_gate_up(dev(Wg, torch.bfloat16), dev(Wu, torch.bfloat16)).contiguous()
-    out = torch.empty(M, F, device="cuda", dtype=torch.bfloat16)
+    buf = torch.full((M + 40, F), 7.0, device="cuda", dtype=torch.bfloat16)
+    out = buf[:M]
     K2.linear(K2.KREA2_EPI_SWIGLU, dev(A, torch.bfloat16), Wgu, out)
     K2.check_device_error()
+    assert torch.all(buf[M:] == 7.0).item()
     ref = O.silu(A @ Wg.T) * (A @ Wu.T)
     assert rel_err(host(out), ref) < 8e-3
 
 
-@pytest.mark.parametrize("B,S,N,K", [
-    (2, 150, 256, 512),        # ragged rows; a batch boundary inside a 32-row block
-    (5, 20, 256, 128),         # one 32-row block spans three batch rows
-    (2, 4608, 6144, 16384),    # the backbone's down projection at the 1024^2 CFG shape
+@pytest.mark.parametrize("B,S,N,K,goff", [
+    (2, 150, 256, 512, 0),        # ragged rows; a batch boundary inside a 32-row block
+    (2, 150, 256, 512, 1),        # the same with gate rows off 16-byte alignment (scalar gate loads)
+    (5, 20, 256, 128, 0),         # one 32-row block spans three batch rows
+    (1, 60, 384, 64, 0),          # one ragged row tile: 32-row blocks partly and wholly past M
+    (2, 4608, 6144, 16384, 0),    # the backbone's down projection at the 1024^2 CFG shape
 ])
-def test_linear_gated_residual(K2, B, S, N, K):
+def test_linear_gated_residual(K2, B, S, N, K, goff):
     M = B * S
     A, W = _bf((M, K), 6), _bf((N, K), 7, K ** -0.5)
     h0 = np.random.default_rng(8).standard_normal((M, N)).astype(np.float32)
-    mod = np.random.default_rng(9).standard_normal((B, 6, N)).astype(np.float32)
-    h = dev(h0, torch.float32)
+    mod = np.random.default_rng(9).standard_normal((B, 6, N + 1)).astype(np.float32)
+    # h is the first M rows of a buffer with 40 more sentinel rows, which must stay untouched
+    hbuf = dev(np.concatenate([h0, np.full((40, N), 7.0, np.float32)]), torch.float32)
+    h = hbuf[:M]
     modd = dev(mod, torch.float32)
-    # gate = modulation chunk 2 of each batch row: base at offset 2N, batch stride 6N
-    K2.linear(K2.KREA2_EPI_RESID, dev(A, torch.bfloat16), dev(W, torch.bfloat16), h, gate=modd.view(-1)[2 * N:],
-              rows_per_batch=S, gate_stride=6 * N)
+    # gate = modulation chunk 2 of each batch row (shifted by goff): base at 2(N+1) + goff, batch
+    # stride 6(N+1); the odd stride and offset keep gate rows off 16-byte alignment when goff = 1
+    W1 = N + 1
+    K2.linear(K2.KREA2_EPI_RESID, dev(A, torch.bfloat16), dev(W, torch.bfloat16), h,
+              gate=modd.view(-1)[2 * W1 + goff:], rows_per_batch=S, gate_stride=6 * W1)
     K2.check_device_error()
     acc = (A @ W.T).astype(np.float64)
-    gate = np.repeat(mod[:, 2], S, axis=0)
+    gate = np.repeat(mod[:, 2, goff:goff + N], S, axis=0)
     ref_delta = gate * acc
     assert rel_err(host(h) - h0, ref_delta) < 1e-3
+    assert torch.all(hbuf[M:] == 7.0).item()
+
+
+def test_linear_gated_residual_unaligned_out_rejected(K2):
+    """The residual is updated by TMA reduce-adds, which need a 16-byte aligned fp32 output."""
+    M, N, K = 64, 128, 64
+    A, W = _bf((M, K), 6), _bf((N, K), 7, K ** -0.5)
+    buf = torch.zeros(M * N + 1, device="cuda", dtype=torch.float32)
+    h = buf[1:].view(M, N)
+    gate = torch.ones(N, device="cuda", dtype=torch.float32)
+    with pytest.raises(K2.Krea2Error):
+        K2.linear(K2.KREA2_EPI_RESID, dev(A, torch.bfloat16), dev(W, torch.bfloat16), h, gate=gate,
+                  rows_per_batch=M, gate_stride=0)
+    K2.check_device_error()
+    assert torch.count_nonzero(buf).item() == 0
 
 
 @pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, 8e-3), (torch.float32, 1e-5)])

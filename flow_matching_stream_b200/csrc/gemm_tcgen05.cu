@@ -47,8 +47,8 @@ struct GemmCfg {
   static constexpr int B_BYTES = BN * BK * 2;   // 32 KB (BN=256) or 16 KB (BN=128)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  // Epilogue staging per warp: two 4 KB swizzled 32x32 fp32 boxes (residual), or one padded
-  // 32x33 fp32 tile (the other epilogues), at 8 KB spacing.
+  // Epilogue staging per warp: two 4 KB swizzled 32x64 bf16 boxes (TMA-store epilogues), or one
+  // padded 32x33 fp32 tile (residual and row-mapped epilogues), at 8 KB spacing.
   static constexpr int EPI_WARP_BYTES = 8192;
   static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;  // + alignment slack
@@ -69,8 +69,8 @@ struct TileMap {
   }
 };
 
-// The TMA epilogues hand each warp's 32 rows to the TMA unit through boxes in shared memory:
-// 32 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle, so 16-byte chunk j of box
+// The bf16 epilogues hand each warp's 32 rows to the TMA unit through boxes in shared memory:
+// 32 rows x 128 bytes (64 bf16 columns), 128-byte swizzle, so 16-byte chunk j of box
 // row r sits at position j ^ (r & 7) and a warp's row-wise 16-byte stores spread over all banks.
 // Rows and columns outside the output are clipped by the tensor map. Each warp owns two boxes
 // and alternates between them; a box is rewritten only once the TMA operation issued from it two
@@ -359,49 +359,47 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           }
         }
       } else {  // EPI_RESID: h[row, col] += gate[b, col] * acc
-        // Each thread scales its row of a 32-column chunk by the gate of its batch row and
-        // writes it into a 32x32 fp32 box; one lane hands the box to the TMA unit as a
-        // reduce-add into h. The read-modify-write of the residual then runs in L2, and the
-        // epilogue never waits on loads of h. The batch row of a ragged last tile's rows is
-        // clamped to M - 1 (an in-bounds gate; those rows are clipped by the tensor map).
+        // A plain read-modify-write of h through L1/L2, not a TMA reduce-add: h is also written
+        // by plain stores (img_in, the text rows, the caller), and in one launch sequence a TMA
+        // reduce-add of this epilogue returned the value h held before the img_in kernel, several
+        // launches earlier in the same stream. After tcgen05.ld each thread holds one row of a
+        // 32-column chunk; row-by-row global accesses would touch 32 cache lines per warp access,
+        // so the warp transposes its 32x32 block through a padded shared tile and walks the rows:
+        // each access is one 128-byte line, and 16 rows of loads are in flight before any store.
+        // Lane i knows the batch row of tile row row0 + i (clamped to M - 1, so that rows of the
+        // ragged last tile read an in-bounds gate; their results are never stored).
+        float* xp = reinterpret_cast<float*>(xpk);
         const int my_b = min(row0 + lane, p.M - 1) / p.rows_per_batch;
-        const float* grow = p.gate + (size_t)my_b * p.gate_stride + (size_t)nt * BN;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
-          uint8_t* box = boxes.next(lane);
-          if (p.gate_vec4) {
-            const float4* g4 = reinterpret_cast<const float4*>(grow + c * 32);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 g = __ldg(g4 + j);
-              box_put16(box, lane, j,
-                        make_uint4(__float_as_uint(v[4 * j] * g.x), __float_as_uint(v[4 * j + 1] * g.y),
-                                   __float_as_uint(v[4 * j + 2] * g.z), __float_as_uint(v[4 * j + 3] * g.w)));
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float* gj = grow + c * 32 + 4 * j;
-              box_put16(box, lane, j,
-                        make_uint4(__float_as_uint(v[4 * j] * __ldg(gj)), __float_as_uint(v[4 * j + 1] * __ldg(gj + 1)),
-                                   __float_as_uint(v[4 * j + 2] * __ldg(gj + 2)),
-                                   __float_as_uint(v[4 * j + 3] * __ldg(gj + 3))));
-            }
-          }
-          fence_proxy_async_smem();
+          for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = v[e];
           __syncwarp();
-          if (lane == 0 && rows_in) {  // a 32-row block wholly past M (ragged last tile) adds nothing
-            tma_reduce_add_2d(&tmC, box, nt * BN + c * 32, row0);
-            bulk_commit_group();
+          const int col = nt * BN + c * 32 + lane;
+#pragma unroll 1
+          for (int i0 = 0; i0 < 32; i0 += 16) {
+            float* hp = reinterpret_cast<float*>(p.out) + (size_t)(row0 + i0) * p.N + col;
+            float hv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) hv[i] = i0 + i < nrows ? hp[(size_t)i * p.N] : 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int bb = __shfl_sync(0xffffffffu, my_b, i0 + i);
+              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (i0 + i < nrows) hp[(size_t)i * p.N] = hv[i];
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
     }
-    // the TMA stores and reduces must be complete (their boxes read, the output written) before
+    // the TMA stores must be complete (their boxes read, the output written) before
     // this CTA's shared memory goes away
     if (lane == 0) bulk_wait_all();
   }
@@ -443,23 +441,6 @@ int make_tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t cols, uint64_t r
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return KREA2_OK;
-}
-
-// Row-major fp32 matrix (rows, cols) as a 2-D TMA map with a 32x32 box and 128-byte swizzle: the
-// residual epilogue's reduce-add target.
-static int make_tmap_f32_2d_box32(CUtensorMap* m, void* ptr, uint64_t cols, uint64_t rows) {
-  auto enc = get_encode_fn();
-  if (!enc) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((cols * 4) & 15))
-    return set_error(KREA2_ERR_ARG, "residual output must be 16-byte aligned with a 16-byte multiple row stride");
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 4};
-  cuuint32_t box[2] = {32, 32};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return set_error(KREA2_ERR_CUDA, "cuTensorMapEncodeTiled (fp32) failed (%d)", (int)r);
   return KREA2_OK;
 }
 
@@ -520,11 +501,12 @@ int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStrea
   rc = make_tmap_bf16_2d(&tb, W, p0.K, p0.w_rows ? p0.w_rows : p0.N, p0.K, BK, BN);
   if (rc) return rc;
   GemmParams p = p0;
-  // the epilogue's TMA target: 32-row boxes of 128 bytes (64 bf16 or 32 fp32 columns)
+  // the bf16 epilogues' TMA target: 32-row boxes of 128 bytes (64 bf16 columns)
   memset(&tc, 0, sizeof(tc));
   if constexpr (EPI == EPI_RESID) {
-    if ((rc = make_tmap_f32_2d_box32(&tc, p.out, p.N, p.M))) return rc;
-    p.gate_vec4 = !(reinterpret_cast<uintptr_t>(p.gate) & 15) && !(p.gate_stride & 3);
+    // plain loads and stores (see the epilogue); the 16-byte rule keeps the API uniform
+    if (reinterpret_cast<uintptr_t>(p.out) & 15)
+      return set_error(KREA2_ERR_ARG, "residual output must be 16-byte aligned");
   } else if constexpr (EPI == EPI_STORE) {
     if ((rc = make_tmap_bf16_2d(&tc, p.out, p.n_store ? p.n_store : p.N, p.M, p.out_ld ? p.out_ld : p.N, 64, 32)))
       return rc;

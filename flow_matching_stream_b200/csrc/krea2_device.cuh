@@ -1,6 +1,6 @@
 // Device helpers for the sm_100a kernels: bf16 packing, mbarriers with bounded waits,
-// TMA tile loads, stores and reduce-adds (no cluster multicast anywhere), tcgen05 (TMEM alloc,
-// MMA, commit, ld).
+// TMA tile loads and stores (no cluster multicast anywhere), tcgen05 (TMEM alloc, MMA, commit,
+// ld).
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -157,15 +157,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
 // Makes this thread's generic-proxy writes to shared memory visible to the TMA unit.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// 2-D tiled reduce-add, this CTA's shared memory -> global: each element of the box is added
-// to global memory (in L2) with the tensor map's type; elements outside the tensor are skipped.
-// Completion is tracked with the issuing thread's bulk async-groups.
-__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, const void* smem_src, int x, int y) {
-  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
-               : "memory");
-}
 // 2-D tiled store, this CTA's shared memory -> global; elements outside the tensor are skipped.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(

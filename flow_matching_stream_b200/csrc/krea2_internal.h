@@ -32,12 +32,11 @@ int take_device_error_attention();
 
 struct GemmParams {
   int M, N, K;              // N = rows of W
-  void* out;                // STORE/SWIGLU: bf16 (M, N) / (M, N/2); RESID: fp32 (M, N), 16-byte aligned
+  void* out;                // STORE/SWIGLU: bf16 (M, N) / (M, N/2); RESID: fp32 (M, N)
   const float* bias;        // STORE: optional per-column bias (N)
   const float* gate;        // RESID: gate[(row / rows_per_batch) * gate_stride + col]
   int rows_per_batch;       // RESID: batch of a row; QKV: sequence length S (position = row % S)
   long long gate_stride;
-  int gate_vec4;            // RESID: gate rows 16-byte aligned (filled by the launcher)
   // QKV: columns [q heads (HD) | k heads (KVD) | v | gate]; q/k heads (128 wide) are
   // RMS-normalised with (1 + qw / kw) and rotated with the RoPE tables of the row's position.
   const float* qw;

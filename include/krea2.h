@@ -30,10 +30,10 @@
  *     before anything is launched. KREA2_ERR_CUDA reports a launch failure.
  *     Kernels that wait on barriers bound every wait; an expired wait sets a device error
  *     word that krea2_check_device_error() reports as KREA2_ERR_TIMEOUT.
- *   - Alignment: the bf16 tensor-core paths move their matrix operands, outputs and the fp32
- *     residual with TMA, which needs 16-byte aligned base addresses (cudaMalloc and torch
- *     allocations are 256-byte aligned). A misaligned pointer there returns KREA2_ERR_ARG
- *     before anything is launched.
+ *   - Alignment: the bf16 tensor-core paths move their matrix operands and bf16 outputs with
+ *     TMA, which needs 16-byte aligned base addresses (cudaMalloc and torch allocations are
+ *     256-byte aligned); the fp32 residual is held to the same rule. A misaligned pointer
+ *     there returns KREA2_ERR_ARG before anything is launched.
  *   - text_mask: uint8 (B, T), 1 = valid text token, 0 = padding; NULL means all valid
  *     ([API] encoder_attention_mask). Padding only removes keys: padded text rows are still
  *     computed as queries, and image keys are always valid.
@@ -263,10 +263,8 @@ int krea2_modulated_rmsnorm(const Krea2Dims* dims, int B, int S, int dtype,
  *             out[r, c] += gate[(r / rows_per_batch) * gate_stride + c] * (A·Wᵀ)[r, c].
  *             (gate_stride = 6C for a modulation chunk; 0 broadcasts one vector.)
  *   bf16 path: Nw % 128 == 0, K % 64 == 0, M >= 1; gate/rows_per_batch used by RESID only.
- *             A, W and out must be 16-byte aligned: KREA2_ERR_ARG otherwise. RESID
- *             rounds the product gate * (A·Wᵀ) to fp32 and then adds it to out in L2 (a TMA
- *             reduce-add); each element is updated by exactly one tile, so results are
- *             deterministic. */
+ *             A, W and out must be 16-byte aligned: KREA2_ERR_ARG otherwise. Each output
+ *             element is written by exactly one thread, so results are deterministic. */
 enum { KREA2_EPI_STORE = 0, KREA2_EPI_SWIGLU = 1, KREA2_EPI_RESID = 2 };
 int krea2_linear(int dtype, int epilogue, int M, int Nw, int K,
                  const void* A, const void* W, void* out,

@@ -100,18 +100,22 @@ __global__ void from_f32_kernel(const float* __restrict__ in, long n, void* __re
 }
 
 // ----------------------------------------------------------------------------- modulated RMSNorm
-// One CTA per output row; C % 4 == 0; 256 threads, float4 loads of the fp32 residual.
+// One CTA per output row; C % 4 == 0; 256 threads, float4 loads of the fp32 residual. NV float4
+// per thread hold the row between the two passes: NV = C / 1024 rounded up (6 for C = 6144), so
+// that no registers are reserved for columns the row does not have.
 // Output row r reads residual row (r / rows) * S_in + row0 + r % rows (the identity for the block
 // norms; the image rows for the final layer) and batch b = r / rows picks the modulation vectors.
-template <bool OUT_BF16>
-__global__ void __launch_bounds__(256) mod_rmsnorm_kernel(ModNormArgs a) {
+// Rows in flight set the bandwidth of this one-pass-over-HBM kernel: the launch bounds keep the
+// registers low enough for 6, 5 or 4 resident CTAs per SM as NV grows (NV = 5, 6 spill 16 bytes).
+template <bool OUT_BF16, int NV>
+__global__ void __launch_bounds__(256, NV <= 4 ? 6 : NV <= 6 ? 5 : 4) mod_rmsnorm_kernel(ModNormArgs a) {
   const long row = blockIdx.x;
   const int C = a.C;
   const int b = (int)(row / a.rows);
   const long in_row = (long)b * a.S_in + a.row0 + row % a.rows;
   const int C4 = C >> 2;
   const float4* x4 = reinterpret_cast<const float4*>(a.h + in_row * C);
-  constexpr int MAXV = 8;  // up to C = 8192
+  constexpr int MAXV = NV;
   float4 xv[MAXV];
   float ss = 0.f;
 #pragma unroll
@@ -601,8 +605,18 @@ int launch_to_dtype(const float* in, long n, void* out, bool out_bf16, cudaStrea
 int launch_mod_rmsnorm_rows(const ModNormArgs& a, cudaStream_t stream) {
   const long rows = (long)a.B * a.rows;
   if (rows == 0) return KREA2_OK;
-  if (a.out_bf16) mod_rmsnorm_kernel<true><<<(unsigned)rows, 256, 0, stream>>>(a);
-  else mod_rmsnorm_kernel<false><<<(unsigned)rows, 256, 0, stream>>>(a);
+  const int nv = (a.C / 4 + 255) / 256;  // C <= 8192 (check_dims)
+  switch (nv) {
+#define KREA2_NORM_NV(V)                                                                  \
+  case V:                                                                                 \
+    if (a.out_bf16) mod_rmsnorm_kernel<true, V><<<(unsigned)rows, 256, 0, stream>>>(a);   \
+    else mod_rmsnorm_kernel<false, V><<<(unsigned)rows, 256, 0, stream>>>(a);             \
+    break;
+    KREA2_NORM_NV(1) KREA2_NORM_NV(2) KREA2_NORM_NV(3) KREA2_NORM_NV(4)
+    KREA2_NORM_NV(5) KREA2_NORM_NV(6) KREA2_NORM_NV(7) KREA2_NORM_NV(8)
+#undef KREA2_NORM_NV
+    default: return set_error(KREA2_ERR_ARG, "modulated RMSNorm supports C <= 8192");
+  }
   return check_launch("mod_rmsnorm");
 }
 

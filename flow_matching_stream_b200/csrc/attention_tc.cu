@@ -146,10 +146,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   __shared__ int n_tiles;
   __shared__ int cta_kmin;  // PREFIX: smallest key_end of this CTA's queries (keys below it need no row mask)
   __shared__ uint16_t tiles[MAX_TILES];
-  __shared__ __align__(8) uint64_t ex_bar[4];   // per lane quarter: both halves posted their row max
-  __shared__ __align__(8) uint64_t fin_bar[4];  // per lane quarter: both halves posted their row sum
-  __shared__ float red_max[2][2][128];  // [tile parity][score half][row]: the two halves' row maxima
-  __shared__ float red_l[2][128];       // [score half][row]: partial row sums at the end
 
   constexpr int QPOS = 128 / G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -214,10 +210,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
     mbar_init(&drain_bar, 1);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(&ex_bar[q], 64);
-      mbar_init(&fin_bar[q], 64);
-    }
     abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
@@ -331,15 +323,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       }
     }
   } else {
-    // ---- softmax warps 2..9: tile row r = 32 * quarter + lane holds head j*G + r / QPOS at
-    // position p0 + r % QPOS. Warps w and w+4 share a TMEM lane quarter (the same rows) and split
-    // each row's 64 scores: half 0 takes keys [0, 32) of the tile, half 1 keys [32, 64). They
-    // exchange the row max through shared memory; each keeps its own partial row sum and its
-    // half of the output columns.
+    // ---- softmax warps 2..9. Warps w and w + 4 share TMEM lane quarter w & 3; warp w takes its
+    // first 16 lanes, w + 4 the last 16. Within a warp, threads t and t + 16 hold the same row
+    // (tile row r holds head j*G + r / QPOS at position p0 + r % QPOS) and split its 64 scores:
+    // half 0 takes keys [0, 32) of the tile, half 1 keys [32, 64). The two halves meet by warp
+    // shuffle: the row max, the rescale decision and the final row sum need no shared memory and
+    // no barrier, and each thread keeps its half of the row's output columns.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int sub = (warp - 2) >> 2;
+    const int half = lane >> 4;
+    const int r = quarter * 32 + sub * 16 + (lane & 15);
+    const uint32_t lane_off = (uint32_t)(quarter * 32 + sub * 16) << 16;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -351,15 +345,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
     constexpr int HK = KT / 2;  // scores per thread and tile
     for (int i = 0; i < n && ok; ++i) {
       const int sb = i & 1;
-      if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
+      // waits are made warp-uniform: the shuffles below need every lane
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i >> 1) & 1, abort))) { ok = false; break; }
       tc_fence_after();
       const int t0 = tiles[i] * KT;
       const int k0 = t0 + half * HK;  // first key of this thread's half
       const uint32_t sbase = tmem + lane_off + sb * KT;
       float v[HK];
-      tmem_ld32(sbase + half * HK, v);
+      tmem_ld32_pair<HK>(sbase, v);
       if ((t0 < p.T && p.text_mask) || (t0 + KT > p.S)) {  // warp-uniform: only partial tiles mask
-        const uint32_t vm = __ballot_sync(0xffffffffu, key_valid(p, b, k0 + lane));
+        const uint32_t vm0 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + lane));
+        const uint32_t vm1 = __ballot_sync(0xffffffffu, key_valid(p, b, t0 + HK + lane));
+        const uint32_t vm = half ? vm1 : vm0;
 #pragma unroll
         for (int e = 0; e < HK; ++e)
           if (!((vm >> e) & 1u)) v[e] = -INFINITY;
@@ -372,7 +369,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
             if (e >= lim) v[e] = -INFINITY;
         }
       }
-      // half-row max: chain k takes v[k], v[k+4], ..., v[k+28] with three-input maxes
+      // half-row max: chain k takes v[k], v[k+4], ..., v[k+28] with three-input maxes; the
+      // other half's max comes from lane t ^ 16
       static_assert(HK == 32, "the max chains below cover 32 scores");
       float m4[4];
 #pragma unroll
@@ -382,46 +380,39 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         for (int t = 1; t < 7; t += 2) a = fmax3(a, v[k + 4 * t], v[k + 4 * t + 4]);
         m4[k] = fmaxf(a, v[k + 28]);
       }
-      red_max[i & 1][half][r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      // the arrive also publishes that this half has read its scores: half 1 writes its P over
-      // score columns 16..31, which hold half 0's keys 16..31
-      tc_fence_before();
-      mbar_arrive(&ex_bar[quarter]);
-      // exps against the running max while the partner warp finishes its half
-      uint32_t pk[HK / 2];
-      float rs = exp_tile<HK>(v, sl2, m == -INFINITY ? 0.f : m, pk);
-      if (!mbar_wait(&ex_bar[quarter], i & 1, abort)) { ok = false; break; }
-      tc_fence_after();
-      const float mx = fmaxf(red_max[i & 1][0][r], red_max[i & 1][1][r]);
+      const float hm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      const float mx = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, 16));
       const float mnew = fmaxf(m, mx * sl2);
       const bool grow = mnew > m + 8.0f;  // m = -inf on the first tile
       float alpha = 1.f;
       const bool any_grow = __any_sync(0xffffffffu, grow);
-      if (any_grow) {
-        if (grow) {
-          alpha = ex2(m - mnew);  // 0 on the first tile
-          m = mnew;
-        }
-        rs = exp_tile<HK>(v, sl2, m == -INFINITY ? 0.f : m, pk);
+      if (grow) {
+        alpha = ex2(m - mnew);  // 0 on the first tile
+        m = mnew;
       }
+      uint32_t pk[HK / 2];
+      const float rs = exp_tile<HK>(v, sl2, m == -INFINITY ? 0.f : m, pk);
       l = l * alpha + rs;
-      tmem_st16(sbase + half * (HK / 2), pk);  // P_i (bf16 pairs) over the tile's first 32 columns
+      // P_i (bf16 pairs) over the tile's first 32 columns: half 0 writes columns [0, 16), half 1
+      // [16, 32). They overlay scores of this warp's own rows only, all read by the load above.
+      tmem_st16_pair<HK / 2>(sbase, pk);
       if (i >= 1 && any_grow) {
         // O must hold P_{i-1} V_{i-1} before it is rescaled. PV_{i-1} is the ((i-1)/2)-th
         // commit on pv_done[(i-1) & 1]; s_full_i already implies PV_{i-2} and earlier are
         // done, and PV_{i+1} needs this tile's P, so the parity below names exactly that phase.
-        if (!mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        {
 #pragma unroll 1
-          for (int c = 0; c < AD / 64; ++c) {
-            float o[32];
-            const uint32_t oa = tmem + lane_off + O_COL + half * (AD / 2) + c * 32;
-            tmem_ld32(oa, o);
+        for (int c = 0; c < AD / 64; ++c) {
+          float o[32];
+          const uint32_t oa = tmem + lane_off + O_COL + c * 32;  // half 1: 64 columns further on
+          tmem_ld32_pair<AD / 2>(oa, o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(oa, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] *= alpha;
+          tmem_st32_pair<AD / 2>(oa, o);
         }
       }
       tmem_wait_st();
@@ -438,17 +429,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
         for (int q = 0; q < AD / 16; ++q) op[q] = make_uint4(0u, 0u, 0u, 0u);
       }
     } else if (ok) {
-      // the output needs the last P V in O and both halves' row sums
-      ok = mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort);
-      if (ok) {
-        tc_fence_after();
-        red_l[half][r] = l;
-        mbar_arrive(&fin_bar[quarter]);
-        ok = mbar_wait(&fin_bar[quarter], 0, abort);
-      }
+      // the output needs the last P V in O
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort));
+      if (ok) tc_fence_after();
     }
+    const float lt = l + __shfl_xor_sync(0xffffffffu, l, 16);  // both halves' row sums
     if (ok && n > 0) {
-      const float lt = red_l[0][r] + red_l[1][r];
       const bool row_ok = pos < p.Sq;
       const long grow_idx = (long)b * p.Sq + pos;
       const float inv_l = lt > 0.f ? 1.f / lt : 0.f;  // a row with no readable key: zeros
@@ -456,7 +442,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
       for (int c = 0; c < AD / 64; ++c) {
         const int col = half * (AD / 2) + c * 32;
         float o[32];
-        tmem_ld32(tmem + lane_off + O_COL + col, o);
+        tmem_ld32_pair<AD / 2>(tmem + lane_off + O_COL + c * 32, o);
         if (row_ok) {
           const uint4* gp = reinterpret_cast<const uint4*>(p.gate + grow_idx * p.g_stride + h * AD + col);
           uint4* op = reinterpret_cast<uint4*>(p.out + grow_idx * p.HD + h * AD + col);

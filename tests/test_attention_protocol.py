@@ -6,9 +6,15 @@ tensor pipe and eight softmax warps (two per TMEM lane quarter) through mbarrier
 * ``s_full[i & 1]``: committed after S_i = Q K_i^T;
 * ``p_full[i & 1]``: all softmax warps wrote P_i over their scores;
 * ``pv_done[i & 1]``: committed after O += P_i V_i;
-* ``ex_bar[q]``: the two halves of lane quarter q exchanged their row maxima;
 * ``k_full``/``k_empty`` and ``v_full``/``v_empty``: the two-stage K and V rings the TMA
   producer fills (K tile i+1 is loaded before V tile i).
+
+Each softmax warp owns 16 rows (lanes) of its quarter, and both halves of each row's scores sit
+in that warp (threads t and t + 16): it reads its rows' scores with one warp-collective load
+and writes P over them, so the halves meet by shuffle, without a barrier. The model also keeps
+the kernel's earlier layout ("columns"), in which the two warps of a quarter split every row's
+columns and exchanged their row maxima through ``ex_bar[q]``: half 1's P lands on scores that
+half 0 reads, so that layout needs the exchange.
 
 This file restates those roles as Python generators and runs them under many random
 interleavings. An mbarrier wait on parity P passes when the number of completed phases has the
@@ -26,8 +32,8 @@ run. Checked invariants:
 * at the end every P·V has run, in order.
 
 Three negative controls must fail: the same model with a single p_full barrier (the protocol
-before consecutive tiles were split across two barriers), one whose softmax warps skip the max
-exchange, and one that frees V stages after QK^T instead of after P·V.
+before consecutive tiles were split across two barriers), the column layout with its max
+exchange skipped, and one that frees V stages after QK^T instead of after P·V.
 """
 import random
 
@@ -41,7 +47,8 @@ KV_STAGES = 2
 
 
 class Model:
-    def __init__(self, n_tiles: int, grows, split_p_full: bool, exchange: bool = True, early_v_release: bool = False):
+    def __init__(self, n_tiles: int, grows, split_p_full: bool, exchange: bool = True, early_v_release: bool = False,
+                 layout: str = "rows"):
         self.n = n_tiles
         self.grows = grows  # grows[(quarter, tile)]: the quarter's rows rescale O at that tile
         self.s_full = [Barrier(1), Barrier(1)]
@@ -49,7 +56,8 @@ class Model:
         nb = 2 if split_p_full else 1
         self.p_full = [Barrier(N_WARPS) for _ in range(nb)]
         self.split = split_p_full
-        self.exchange = exchange          # False: a warp does not wait for its partner's max
+        self.layout = layout              # "rows": warp owns 16 rows; "columns": warps split each row
+        self.exchange = exchange          # columns layout, False: a warp skips its partner's max
         self.early_v_release = early_v_release  # True: V stages freed after QK^T, not after P·V
         self.ex_bar = [Barrier(N_HALVES) for _ in range(N_QUARTERS)]
         self.fifo = []                    # issued tensor-pipe work, executed in order
@@ -174,15 +182,22 @@ class Model:
             if self.s_buf[i & 1] != i:
                 raise Violation(f"warp ({q},{h}) read buffer {i & 1} holding tile {self.s_buf[i & 1]}, not {i}")
             self.read_scores.add((i, q, h))
-            self.red_max[(i & 1, q, h)] = i
-            self.ex_bar[q].arrive()
-            yield
-            while self.exchange and not self.ex_bar[q].test_parity(i & 1):
+            if self.layout == "rows":
+                # one collective load read every score of this warp's rows; P goes over them
                 yield
-            if self.red_max.get((i & 1, q, 1 - h)) != i:
-                raise Violation(f"warp ({q},{h}) read its partner's max of tile {self.red_max.get((i & 1, q, 1 - h))}")
-            if (i, q, 1 - h) not in self.read_scores:
-                raise Violation(f"warp ({q},{h}) wrote P_{i} before its partner read the scores under it")
+                if (i, q, h) not in self.read_scores:
+                    raise Violation(f"warp ({q},{h}) wrote P_{i} over scores it did not read")
+            else:
+                self.red_max[(i & 1, q, h)] = i
+                self.ex_bar[q].arrive()
+                yield
+                while self.exchange and not self.ex_bar[q].test_parity(i & 1):
+                    yield
+                if self.red_max.get((i & 1, q, 1 - h)) != i:
+                    raise Violation(f"warp ({q},{h}) read its partner's max of tile "
+                                    f"{self.red_max.get((i & 1, q, 1 - h))}")
+                if (i, q, 1 - h) not in self.read_scores:
+                    raise Violation(f"warp ({q},{h}) wrote P_{i} before its partner read the scores under it")
             self.p_written[i & 1][(q, h)] = i
             yield
             if i >= 1 and self.grows[(q, i)]:
@@ -202,10 +217,10 @@ class Model:
 
 
 def run(n_tiles: int, seed: int, split_p_full: bool = True, exchange: bool = True, early_v_release: bool = False,
-        max_steps: int = 200_000):
+        max_steps: int = 200_000, layout: str = "rows"):
     rng = random.Random(seed)
     grows = {(q, i): rng.random() < 0.3 for q in range(N_QUARTERS) for i in range(n_tiles)}
-    m = Model(n_tiles, grows, split_p_full, exchange, early_v_release)
+    m = Model(n_tiles, grows, split_p_full, exchange, early_v_release, layout)
     roles = [m.producer(), m.mma_thread()] + [m.softmax_warp(q, h) for q in range(N_QUARTERS)
                                               for h in range(N_HALVES)]
     schedule(rng, roles, [m.tensor_pipe(), m.tma_engine()], max_steps)
@@ -219,6 +234,12 @@ def test_protocol_holds_under_random_interleavings(n_tiles):
         assert m.pv_applied == list(range(n_tiles))
 
 
+def test_the_column_layout_holds_with_its_max_exchange():
+    for seed in range(200):
+        m = run(5, seed, layout="columns")
+        assert m.pv_applied == list(range(5))
+
+
 def test_a_single_p_full_barrier_lets_a_fast_quarter_complete_a_slow_quarters_phase():
     failures = 0
     for seed in range(400):
@@ -229,12 +250,12 @@ def test_a_single_p_full_barrier_lets_a_fast_quarter_complete_a_slow_quarters_ph
     assert failures > 0
 
 
-def test_writing_p_without_the_max_exchange_is_caught():
-    # the exchange is also what keeps half 1's P off half 0's unread scores
+def test_the_column_layout_without_the_max_exchange_is_caught():
+    # there the exchange is also what keeps half 1's P off half 0's unread scores
     failures = 0
     for seed in range(200):
         try:
-            run(4, seed, exchange=False)
+            run(4, seed, exchange=False, layout="columns")
         except Violation:
             failures += 1
     assert failures > 0

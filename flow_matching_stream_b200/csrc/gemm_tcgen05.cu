@@ -14,12 +14,14 @@
 //               signals a finished accumulator.
 //   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane), reads 32 columns
 //               at a time with tcgen05.ld and applies the fused epilogue, while the MMA warp
-//               already accumulates the next tile into the other TMEM buffer. The residual,
-//               plain and q/k/v/gate epilogues pass each warp's 32 rows through a padded
-//               shared tile, so that global accesses run in whole 128-byte row segments (the
-//               SwiGLU epilogue, with half the output bytes, measured no gain from it).
-// Tiles are visited in groups of row tiles (sized so the group's A tiles stay in L2) so that
-// concurrently running CTAs share W and A tiles through L2.
+//               already accumulates the next tile into the other TMEM buffer. The bf16
+//               epilogues (plain, SwiGLU, q/k/v/gate) write each warp's 32 rows into swizzled
+//               shared-memory boxes that TMA stores; the fp32 residual and the row-mapped
+//               output pass through a padded shared tile so that global accesses run in whole
+//               128-byte row segments.
+// Tiles are visited in raster groups of row tiles, sized so that one wave of tiles reads about
+// as many A bytes as W bytes per K step and so that concurrently running CTAs share A and W
+// tiles through L2.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

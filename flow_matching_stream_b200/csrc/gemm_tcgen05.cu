@@ -475,8 +475,8 @@ namespace {
 // Row tiles per raster group. The persistent CTAs run about `sms` consecutive tiles at once: r
 // row tiles by c = sms / r column tiles of one group. Per K step that wave reads r*BM rows of A
 // and c*BN rows of W, which is least at r = sqrt(sms * BN / BM) (18 for BN = 256 on 148 SMs);
-// fewer rows stream W from HBM once per wave (down, K = 16384, took 6 by the L2 rule alone).
-// The row tiles are then split into groups of equal size.
+// with much fewer rows, each wave streams nearly all of W from HBM. The row tiles are then split
+// into groups of equal size.
 int group_rows(int tiles_m, int K, int BN, int sms) {
   const int by_l2 = (int)(GROUP_A_BYTES / ((size_t)BM * K * 2));
   const int by_wave = (int)std::ceil(std::sqrt((double)sms * BN / BM));

@@ -133,6 +133,24 @@ def test_modulated_rmsnorm(K2, dtype, tol, chunk, B, S):
     assert rel_err(host(out).reshape(B, S, d.C), ref) < tol
 
 
+@pytest.mark.parametrize("C", [128, 1152, 2560, 4096, 5120, 7168, 8192])
+def test_modulated_rmsnorm_widths(K2, C):
+    """The norm kernel keeps ceil(C / 1024) float4 per thread in registers: one instantiation
+    per width class, 1 to 8 (C = 6144, the model's, is covered above)."""
+    d = KI.Dims(C=C, H=C // 128, Hkv=C // 128, D=128, F=256)
+    B, S = 2, 37
+    h = KI.residual(d, B, S)
+    temb = KI.temb(d, B)
+    table = KI._normal(0, (98, 1), (6, C), 0.1)
+    nw = KI._normal(0, (98, 2), (C,), 0.1)
+    out = torch.empty(B * S, C, device="cuda", dtype=torch.float32)
+    K2.modulated_rmsnorm(d, B, S, dev(h.reshape(B * S, C), torch.float32), dev(nw, torch.float32),
+                         dev(temb, torch.float32), dev(table, torch.float32), 3, out)
+    mod = O.modulation(temb, table)
+    ref = (1 + mod[:, 3][:, None]) * O.rms_norm(h, nw, d.eps) + mod[:, 4][:, None]
+    assert rel_err(host(out).reshape(B, S, C), ref) < TOL_F32
+
+
 @pytest.mark.parametrize("dims,dtype,tol", [(KI.FULL, torch.bfloat16, 2e-3), (KI.TINY, torch.float32, TOL_F32)])
 def test_time_embed(K2, dims, dtype, tol):
     mw_h = KI.model_weights(dims)

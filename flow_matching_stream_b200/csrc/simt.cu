@@ -186,11 +186,13 @@ __device__ __forceinline__ float gelu_tanh_f(float x) {
 }
 
 // out[b, n] = act(sum_k x[b, k] W[n, k] + bias[n]); one warp per output feature, all batch rows.
-template <bool W_BF16, bool GELU>
+// MAXB accumulators per lane, sized to the batch (1, 2, 4 or 8 at a time), so that with the
+// model's batch of one or two the K loop can keep four 16-byte weight loads in flight per lane:
+// the weights stream from HBM once and this is a bandwidth-bound GEMV.
+template <bool W_BF16, bool GELU, int MAXB>
 __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __restrict__ x, const void* __restrict__ W,
                                                              const float* __restrict__ bias, int B, int N, int K,
                                                              float* __restrict__ out) {
-  constexpr int MAXB = 8;
   const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (n >= N) return;
@@ -198,6 +200,7 @@ __global__ void __launch_bounds__(256) small_m_linear_kernel(const float* __rest
     float acc[MAXB];
 #pragma unroll
     for (int b = 0; b < MAXB; ++b) acc[b] = 0.f;
+#pragma unroll 4
     for (int k = lane * 8; k < K; k += 256) {
       float wv[8];
       if (W_BF16) {
@@ -640,13 +643,21 @@ int launch_time_embed(const Krea2Dims* d, int B, bool w_bf16, const float* t, co
   if (rc) return rc;
   auto lin = [&](const float* x, const void* W, const float* bias, int N, int K, float* out, bool gelu) {
     dim3 grid((N + 7) / 8);
-    if (w_bf16) {
-      if (gelu) small_m_linear_kernel<true, true><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);
-      else small_m_linear_kernel<true, false><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);
-    } else {
-      if (gelu) small_m_linear_kernel<false, true><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);
-      else small_m_linear_kernel<false, false><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);
-    }
+#define KREA2_GEMV(MB)                                                                                   \
+  do {                                                                                                   \
+    if (w_bf16) {                                                                                        \
+      if (gelu) small_m_linear_kernel<true, true, MB><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);   \
+      else small_m_linear_kernel<true, false, MB><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);       \
+    } else {                                                                                             \
+      if (gelu) small_m_linear_kernel<false, true, MB><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);  \
+      else small_m_linear_kernel<false, false, MB><<<grid, 256, 0, stream>>>(x, W, bias, B, N, K, out);      \
+    }                                                                                                    \
+  } while (0)
+    if (B <= 1) KREA2_GEMV(1);
+    else if (B <= 2) KREA2_GEMV(2);
+    else if (B <= 4) KREA2_GEMV(4);
+    else KREA2_GEMV(8);
+#undef KREA2_GEMV
     return check_launch("time_linear");
   };
   if ((rc = lin(e, w->t1_w, w->t1_b, C, td, scratch, true))) return rc;

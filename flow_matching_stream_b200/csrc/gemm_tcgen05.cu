@@ -41,7 +41,13 @@ constexpr int BK = 64;
 // (128 x K bf16 each) within about 24 MB of L2, so W streams from HBM once per group pass, and
 // at least as many as make one wave of tiles read about as many A bytes as W bytes per K step.
 constexpr size_t GROUP_A_BYTES = 24ull << 20;
-constexpr int GEMM_THREADS = 192;
+// Epilogue warps: 8 for the residual (two per TMEM lane quarter, each on half the tile's
+// columns), 4 for the others. The residual's read-modify-write of h is bound by the loads in
+// flight; with 4 warps it took longer per tile than to_out's mainloop (K = 6144).
+template <int EPI>
+constexpr int epi_warps() { return EPI == EPI_RESID ? 8 : 4; }
+template <int EPI>
+constexpr int gemm_threads() { return 64 + 32 * epi_warps<EPI>(); }
 
 template <int BN>
 struct GemmCfg {
@@ -107,7 +113,7 @@ __device__ __forceinline__ void store_box_bf16(uint8_t* box, const uint32_t* pk,
 }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(gemm_threads<EPI>(), 1)
     gemm_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmC, GemmParams p) {
   using Cfg = GemmCfg<BN>;
@@ -134,7 +140,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], 32 * epi_warps<EPI>());
     }
     mbar_init(&drain_bar, 1);
     abort_flag = 0;
@@ -223,8 +229,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       }
     }
   } else {
-    // epilogue warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
+    // epilogue warps 2.. -> TMEM lane quarters 2, 3, 0, 1 (2, 3, 0, 1 again for the residual's
+    // second four warps, which take the other half of the columns)
     const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;
     EpiBoxes boxes{base + STAGES * Cfg::STAGE_BYTES + (warp - 2) * Cfg::EPI_WARP_BYTES, 0};
     int local = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++local) {
@@ -366,18 +374,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         // reduce-add of this epilogue returned the value h held before the img_in kernel, several
         // launches earlier in the same stream. After tcgen05.ld each thread holds one row of a
         // 32-column chunk; row-by-row global accesses would touch 32 cache lines per warp access,
-        // so the warp transposes its 32x32 block through a padded shared tile and walks the rows:
-        // each access is one 128-byte line, and 16 rows of loads are in flight before any store.
+        // so the warp transposes its 32x32 block through shared memory (XOR-swizzled: element
+        // (row i, column e) at i * 32 + (e ^ i), conflict-free both ways) and walks the rows: each
+        // access is one 128-byte line, and 16 rows of loads are in flight before any store. Warp
+        // part 0 takes the tile's first BN / 2 columns, part 1 the rest.
         // Lane i knows the batch row of tile row row0 + i (clamped to M - 1, so that rows of the
         // ragged last tile read an in-bounds gate; their results are never stored).
-        float* xp = reinterpret_cast<float*>(xpk);
+        float* xp = reinterpret_cast<float*>(base + STAGES * Cfg::STAGE_BYTES) + (warp - 2) * (32 * 32);
         const int my_b = min(row0 + lane, p.M - 1) / p.rows_per_batch;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = part * (BN / 64); c < (part + 1) * (BN / 64); ++c) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) xp[lane * 33 + e] = v[e];
+          for (int e = 0; e < 32; ++e) xp[lane * 32 + (e ^ lane)] = v[e];
           __syncwarp();
           const int col = nt * BN + c * 32 + lane;
 #pragma unroll 1
@@ -389,7 +399,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int bb = __shfl_sync(0xffffffffu, my_b, i0 + i);
-              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 33 + lane];
+              hv[i] += __ldg(p.gate + (size_t)bb * p.gate_stride + col) * xp[(i0 + i) * 32 + (lane ^ (i0 + i))];
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -522,7 +532,7 @@ int launch_gemm_bn(const GemmParams& p0, const void* A, const void* W, cudaStrea
   p.group_m = group_rows(p.tiles_m, p.K, BN, num_sms());
   const int total = p.tiles_m * p.tiles_n;
   const int grid = total < num_sms() ? total : num_sms();
-  kern<<<grid, GEMM_THREADS, Cfg::SMEM_BYTES, stream>>>(ta, tb, tc, p);
+  kern<<<grid, gemm_threads<EPI>(), Cfg::SMEM_BYTES, stream>>>(ta, tb, tc, p);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(KREA2_ERR_CUDA, "gemm launch failed: %s", cudaGetErrorString(e));

@@ -1,12 +1,13 @@
 """A randomized model check of the persistent GEMM kernel's barrier protocol (CPU).
 
 The tcgen05 GEMM (gemm_tcgen05.cu) runs, per CTA, a TMA producer thread, one MMA-issuing
-thread and four epilogue warps over a ring of shared-memory stages and two TMEM accumulators:
+thread and four epilogue warps (eight for the gated residual, two per TMEM lane quarter) over a
+ring of shared-memory stages and two TMEM accumulators:
 
 * ``full[s]`` completes when stage s's TMA loads have landed; ``empty[s]`` is committed after
   the MMAs that read stage s;
 * ``tfull[a]`` is committed after a tile's last MMA into accumulator a; ``tempty[a]``
-  completes when all four epilogue warps have read accumulator a.
+  completes when every epilogue warp has read accumulator a.
 
 The producer waits ``empty`` with the flipped parity (the ring starts empty), the MMA thread
 waits ``tempty`` with the flipped parity (both accumulators start free), as the kernel does.
@@ -19,8 +20,9 @@ tensor pipe, TMA loads that land later) and checks under random interleavings th
 * the MMA starts a tile in an accumulator only after the epilogue of the tile before it
   there has finished.
 
-Negative controls (an empty-barrier wait without the parity flip, and a tempty barrier that
-expects one arrival where four warps arrive) must fail.
+Negative controls must fail: an empty-barrier wait without the parity flip, a tempty barrier
+that expects one arrival where four warps arrive, and one that still expects four where the
+residual's eight arrive.
 """
 import random
 
@@ -28,12 +30,12 @@ import pytest
 
 from protocol_model import Barrier, Violation, schedule
 
-N_EPI = 4
-
-
 class Gemm:
-    def __init__(self, tiles: int, nk: int, stages: int, flip_empty: bool = True, tempty_count: int = N_EPI):
+    def __init__(self, tiles: int, nk: int, stages: int, flip_empty: bool = True, n_epi: int = 4,
+                 tempty_count: int = None):
         self.tiles, self.nk, self.S = tiles, nk, stages
+        self.n_epi = n_epi
+        tempty_count = n_epi if tempty_count is None else tempty_count
         self.full = [Barrier(1) for _ in range(stages)]
         self.empty = [Barrier(1) for _ in range(stages)]
         self.tfull = [Barrier(1), Barrier(1)]
@@ -97,7 +99,7 @@ class Gemm:
             while not self.tempty[a].test_parity(((t >> 1) & 1) ^ 1):
                 yield
             prev = self.acc[a]
-            if prev is not None and self.reads_done.get(prev[0], 0) != N_EPI:
+            if prev is not None and self.reads_done.get(prev[0], 0) != self.n_epi:
                 raise Violation(f"tile {t} claimed accumulator {a} before all epilogue warps read tile {prev[0]}")
             self.acc[a] = (t, 0)
             for kb in range(self.nk):
@@ -131,18 +133,19 @@ class Gemm:
 def run(tiles: int, nk: int, stages: int, seed: int, max_steps: int = 200_000, **kw):
     rng = random.Random(seed)
     g = Gemm(tiles, nk, stages, **kw)
-    roles = [g.producer(), g.mma()] + [g.epilogue(w) for w in range(N_EPI)]
+    roles = [g.producer(), g.mma()] + [g.epilogue(w) for w in range(g.n_epi)]
     schedule(rng, roles, [g.tma_engine(), g.tensor_pipe()], max_steps)
     return g
 
 
+@pytest.mark.parametrize("n_epi", [4, 8])
 @pytest.mark.parametrize("tiles,nk,stages", [(1, 1, 4), (3, 5, 4), (6, 2, 4), (5, 7, 6), (4, 3, 1)])
-def test_protocol_holds_under_random_interleavings(tiles, nk, stages):
+def test_protocol_holds_under_random_interleavings(tiles, nk, stages, n_epi):
     for seed in range(200):
-        run(tiles, nk, stages, seed)
+        run(tiles, nk, stages, seed, n_epi=n_epi)
 
 
-@pytest.mark.parametrize("kw", [dict(flip_empty=False), dict(tempty_count=1)])
+@pytest.mark.parametrize("kw", [dict(flip_empty=False), dict(tempty_count=1), dict(n_epi=8, tempty_count=4)])
 def test_broken_protocols_are_caught(kw):
     # a deadlock counts as a failure too (no progress within the step budget)
     for seed in range(200):

@@ -9,8 +9,8 @@ Euler + CFG update and so keep identical latents, with no further exchange.
 
 This module only orchestrates. `velocity_fn` runs the rank's backbone forward and `step_fn`
 the Euler + CFG update. On GPUs these are the library's krea2_backbone_forward and
-krea2_euler_cfg_step, and the all-gather goes over NCCL on NVLink. No tensor-memory
-multicast or remote-memory TMA is involved.
+krea2_euler_cfg_step, and the all-gather goes over NCCL on NVLink. No kernel reads another
+GPU's memory.
 """
 from __future__ import annotations
 

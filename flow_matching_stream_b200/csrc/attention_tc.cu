@@ -10,7 +10,7 @@
 //   * The 128-row MMA tile stacks the G query heads of KV head j (G = 4 in the Krea 2 block):
 //     row r = QPOS*hl + p holds head G*j+hl at position p0+p, QPOS = 128/G. One K/V tile in
 //     shared memory therefore serves all G heads (K/V are never copied per query head).
-//   * warp 0: TMA producer (Q once; K and V 64-key tiles, 2-stage ring). No cluster multicast.
+//   * warp 0: TMA producer (Q once; K and V 64-key tiles, 2-stage ring), into this CTA's own shared memory.
 //   * warp 1: MMA issuer. S_i = Q K_iᵀ into one of two TMEM score buffers; P_i (bf16, written
 //     back over its own scores) is the TMEM A operand of O += P_i V_i, V being the MN-major B
 //     operand in shared memory.

@@ -8,7 +8,7 @@
 //
 // Design (one CTA per SM, persistent over output tiles):
 //   warp 0      TMA producer: A tile 128x64 and W tile BNx64 per stage, 128-byte swizzle,
-//               STAGES-deep ring guarded by full/empty mbarriers. No cluster multicast.
+//               STAGES-deep ring guarded by full/empty mbarriers, into this CTA's own shared memory.
 //   warp 1      allocates TMEM (2 accumulators x BN fp32 columns) and issues tcgen05.mma
 //               (M=128, N=BN, K=16) from one thread; tcgen05.commit frees smem stages and
 //               signals a finished accumulator.

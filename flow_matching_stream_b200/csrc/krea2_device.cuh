@@ -1,5 +1,5 @@
 // Device helpers for the sm_100a kernels: bf16 packing, mbarriers with bounded waits,
-// TMA tile loads and stores (no cluster multicast anywhere), tcgen05 (TMEM alloc, MMA, commit,
+// TMA tile loads and stores (each CTA loads only into its own shared memory), tcgen05 (TMEM alloc, MMA, commit,
 // ld).
 #pragma once
 #include <cuda_bf16.h>
